@@ -1,0 +1,181 @@
+"""Pins of the oracle's routing, weight-site and grouping steps (CPU only).
+
+Each test checks the oracle against something other than itself: the worked example on the
+frink-models page, a library routine (scipy's softmax), brute force over tiny inputs, or a
+closed-form property that a dropped term, wrong index or transposed operand would break.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import softmax as scipy_softmax
+
+from oracle import moe_ref as ref
+from mixture_experts_decode_gemv_b200.synthetic import LayerConfig
+
+pytestmark = pytest.mark.cpu
+
+
+def cfg_of(**kw):
+    base = dict(name="t", hidden=8, num_experts=6, top_k=2, moe_inter=4)
+    base.update(kw)
+    return LayerConfig(**base)
+
+
+# ---- routed-weight site: the worked example ---------------------------------------------------
+
+def test_routed_slot_worked_example(golden_dir):
+    with open(os.path.join(golden_dir, "routed_slot_worked_example.json")) as f:
+        g = json.load(f)
+    x = np.array(g["x"])
+    xin, w = ref.routed_slot(x, g["w"], False)
+    np.testing.assert_array_equal(xin, g["after_ffn"]["input"])
+    assert w == g["after_ffn"]["weight"]
+    xin, w = ref.routed_slot(x, g["w"], True)
+    np.testing.assert_array_equal(xin, g["before_ffn"]["input"])
+    assert w == g["before_ffn"]["weight"]
+    for arch, flag in g["weight_before_ffn"].items():
+        assert ref.weight_before_ffn(arch) is flag
+
+
+# ---- top-k -------------------------------------------------------------------------------------
+
+def _is_valid_topk(keys, ids, k):
+    """Brute-force definition: the selected set holds the k best (key, -id) pairs and is listed in
+    descending key order with ties to the lower id."""
+    ranked = [(-keys[e], e) for e in range(len(keys))]
+    chosen = sorted(ranked[e] for e in ids)
+    rest = [ranked[e] for e in range(len(keys)) if e not in ids]
+    if len(set(ids)) != k:
+        return False
+    if rest and max(chosen) > min(rest):
+        return False
+    return [ranked[e] for e in ids] == chosen
+
+
+def test_topk_brute_force_with_ties():
+    rng = np.random.default_rng(1)
+    for trial in range(300):
+        E = int(rng.integers(1, 9))
+        k = int(rng.integers(1, E + 1))
+        keys = rng.integers(0, 3, size=E).astype(np.float64)  # many ties
+        ids = ref.select_top_k(keys, k)
+        assert _is_valid_topk(list(keys), ids, k), (keys, ids)
+        # exhaustive: among all k-subsets, the chosen set is the lexicographically best
+        best = max(itertools.combinations(range(E), k),
+                   key=lambda c: sorted(((keys[e], -e) for e in c), reverse=True))
+        assert sorted(ids) == sorted(best)
+
+
+def test_topk_on_sigmoid_equals_topk_on_raw_logits():
+    rng = np.random.default_rng(2)
+    c_raw = cfg_of(routing="sigmoid", select_on_raw_logits=True, norm_topk_prob=False, top_k=3,
+                   num_experts=16)
+    c_sig = c_raw.replace(select_on_raw_logits=False)
+    for _ in range(200):
+        l = rng.standard_normal(16) * 3
+        a = ref.select_top_k(ref.selection_keys(l, c_raw, None), 3)
+        b = ref.select_top_k(ref.selection_keys(l, c_sig, None), 3)
+        assert a == b
+    # and the weights are the sigmoid of the selected logits, un-normalised
+    l = np.array([0.0, 2.0, -1.0, 1.0])
+    ids, w = ref.route_row(l, cfg_of(num_experts=4, top_k=2, routing="sigmoid",
+                                     select_on_raw_logits=True, norm_topk_prob=False), None)
+    assert ids == [1, 3]
+    np.testing.assert_allclose(w, [1 / (1 + math.exp(-2.0)), 1 / (1 + math.exp(-1.0))],
+                               rtol=0, atol=1e-15)
+
+
+def test_biased_selection_unbiased_weights():
+    l = np.array([2.0, 1.0, 0.0, -1.0])
+    bias = np.array([0.0, 0.0, 3.0, 0.0], dtype=np.float32)
+    c = cfg_of(num_experts=4, top_k=2, routing="sigmoid", has_expert_bias=True,
+               norm_topk_prob=True, routed_scaling_factor=2.5)
+    ids, w = ref.route_row(l, c, bias)
+    # the bias moves expert 2 into the set; the unbiased ranking would be [0, 1]
+    assert ids == [2, 0]
+    s2, s0 = 0.5, 1 / (1 + math.exp(-2.0))
+    np.testing.assert_allclose(w, [2.5 * s2 / (s2 + s0), 2.5 * s0 / (s2 + s0)], atol=1e-15)
+    # zero bias reduces to plain sigmoid top-k
+    ids0, w0 = ref.route_row(l, c, np.zeros(4, dtype=np.float32))
+    ids1, w1 = ref.route_row(l, c.replace(has_expert_bias=False), None)
+    assert ids0 == ids1 == [0, 1]
+    np.testing.assert_array_equal(w0, w1)
+
+
+def test_normalised_weights_sum_to_one_then_scale():
+    rng = np.random.default_rng(3)
+    for routing in ("softmax", "sigmoid"):
+        for rsf in (1.0, 2.5):
+            c = cfg_of(num_experts=32, top_k=5, routing=routing, norm_topk_prob=True,
+                       routed_scaling_factor=rsf)
+            for _ in range(50):
+                l = rng.standard_normal(32)
+                _, w = ref.route_row(l, c, None)
+                assert abs(w.sum() - np.float32(rsf)) <= 1e-14 * max(1.0, rsf)
+
+
+def test_softmax_k_equals_E_is_plain_softmax():
+    rng = np.random.default_rng(4)
+    c = cfg_of(num_experts=7, top_k=7, routing="softmax", norm_topk_prob=True)
+    for _ in range(20):
+        l = rng.standard_normal(7) * 2
+        ids, w = ref.route_row(l, c, None)
+        np.testing.assert_allclose(w, scipy_softmax(l)[ids], rtol=1e-14, atol=0)
+        # slot order is descending probability
+        assert list(ids) == list(np.argsort(-l, kind="stable"))
+
+
+def test_softmax_without_norm_is_probability_over_all_experts():
+    rng = np.random.default_rng(5)
+    c = cfg_of(num_experts=12, top_k=3, routing="softmax", norm_topk_prob=False)
+    l = rng.standard_normal(12)
+    ids, w = ref.route_row(l, c, None)
+    np.testing.assert_allclose(w, scipy_softmax(l)[ids], rtol=1e-14, atol=0)
+    assert w.sum() < 1.0
+
+
+def test_top1_normalised_weight_is_one():
+    rng = np.random.default_rng(6)
+    for routing in ("softmax", "sigmoid"):
+        c = cfg_of(num_experts=9, top_k=1, routing=routing, norm_topk_prob=True)
+        _, w = ref.route_row(rng.standard_normal(9), c, None)
+        assert w[0] == 1.0
+
+
+# ---- grouping by expert ------------------------------------------------------------------------
+
+def _counting_sort(flat, E):
+    """Hand-written stable counting sort (independent of numpy's argsort)."""
+    buckets = [[] for _ in range(E)]
+    for p, e in enumerate(flat):
+        buckets[e].append(p)
+    order = [p for b in buckets for p in b]
+    offsets = [0]
+    for b in buckets:
+        offsets.append(offsets[-1] + len(b))
+    return order, offsets
+
+
+def test_grouping_matches_counting_sort():
+    rng = np.random.default_rng(8)
+    for _ in range(200):
+        E = int(rng.integers(1, 20))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        m = int(rng.integers(1, 9))
+        idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(m)])
+        g = ref.group_by_expert(idx, E)
+        order, offsets = _counting_sort(list(idx.ravel()), E)
+        assert list(g["sorted_pairs"]) == order
+        assert list(g["expert_offsets"]) == offsets
+        te = m * k
+        assert g["expert_offsets"][-1] == te
+        tp = g["token_to_perm"]
+        assert list(tp[g["sorted_pairs"]]) == list(range(te))
+        assert list(g["sorted_pairs"][tp]) == list(range(te))
+        active = [e for e in range(E) if offsets[e + 1] > offsets[e]]
+        assert list(g["active"]) == active
+        assert g["active_count"] == len(active) <= min(te, E)
