@@ -1,0 +1,418 @@
+// Host side of the C ABI: argument checks, workspace layout, kernel selection and launches.
+//
+// Every check happens before the first CUDA call that could launch work, so a refused call
+// launches nothing (the serve predicate of metrale "forward_bf16_grouped_decode.rs": the grouped
+// decode launches nothing unless its predicate holds).
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "experts.cuh"
+#include "router.cuh"
+
+using namespace moe;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return MOE_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int check_cfg(const moe_cfg* c, int m) {
+  if (!c) return MOE_ERR_NULL_POINTER;
+  if (m < 1 || m > MOE_MAX_ROWS) return MOE_ERR_BAD_SHAPE;
+  if (c->hidden <= 0 || c->hidden % 8) return MOE_ERR_BAD_SHAPE;
+  if (c->num_experts < 1 || c->num_experts > MOE_MAX_EXPERTS) return MOE_ERR_BAD_SHAPE;
+  if (c->top_k < 1 || c->top_k > MOE_MAX_TOP_K || c->top_k > c->num_experts)
+    return MOE_ERR_BAD_SHAPE;
+  if (c->moe_inter <= 0 || c->moe_inter % 4 || c->shared_inter < 0) return MOE_ERR_BAD_SHAPE;
+  if (c->routing != MOE_ROUTE_SOFTMAX && c->routing != MOE_ROUTE_SIGMOID) return MOE_ERR_BAD_OPTION;
+  auto is01 = [](int v) { return v == 0 || v == 1; };
+  if (!is01(c->norm_topk_prob) || !is01(c->select_on_raw_logits) || !is01(c->has_expert_bias) ||
+      !is01(c->weight_before_ffn))
+    return MOE_ERR_BAD_OPTION;
+  if (c->routing == MOE_ROUTE_SOFTMAX && (c->select_on_raw_logits || c->has_expert_bias))
+    return MOE_ERR_BAD_OPTION;
+  if (c->select_on_raw_logits && c->has_expert_bias) return MOE_ERR_BAD_OPTION;
+  if (!std::isfinite(c->routed_scaling_factor)) return MOE_ERR_BAD_OPTION;
+  if (c->shared_kind < MOE_SHARED_NONE || c->shared_kind > MOE_SHARED_SIGMOID_GATE)
+    return MOE_ERR_BAD_OPTION;
+  if (c->shared_kind != MOE_SHARED_NONE && c->shared_inter <= 0) return MOE_ERR_BAD_SHAPE;
+  if (c->shared_kind == MOE_SHARED_NONE && c->shared_inter != 0) return MOE_ERR_BAD_OPTION;
+  if (c->shared_inter % 4) return MOE_ERR_BAD_SHAPE;
+  if (c->x_dtype != MOE_FMT_F32 && c->x_dtype != MOE_FMT_BF16) return MOE_ERR_BAD_FORMAT;
+  if (c->out_dtype != MOE_FMT_F32 && c->out_dtype != MOE_FMT_BF16) return MOE_ERR_BAD_FORMAT;
+  return MOE_OK;
+}
+
+// k-dimension rule of each format: 16-byte packed rows, whole scale groups.
+bool k_ok(int fmt, int k) {
+  switch (fmt) {
+    case MOE_FMT_F32: return k % 4 == 0;
+    case MOE_FMT_BF16: return k % 8 == 0;
+    case MOE_FMT_Q4_AFFINE_G64: return k % 64 == 0;
+    case MOE_FMT_NVFP4: return k % 32 == 0;
+    default: return false;
+  }
+}
+
+int check_matrix(const moe_matrix& M, int n, int k, int E, MatDev* out) {
+  if (M.format < MOE_FMT_F32 || M.format > MOE_FMT_NVFP4) return MOE_ERR_BAD_FORMAT;
+  if (!k_ok(M.format, k)) return MOE_ERR_BAD_FORMAT;
+  if (!M.packed) return MOE_ERR_NULL_POINTER;
+  if (!aligned(M.packed, 16)) return MOE_ERR_MISALIGNED;
+  const size_t mat_bytes = packed_row_bytes(M.format, k) * (size_t)n;
+  if (E > 1 && (M.expert_stride < (int64_t)mat_bytes || M.expert_stride % 16))
+    return M.expert_stride % 16 ? MOE_ERR_MISALIGNED : MOE_ERR_BAD_SHAPE;
+  size_t scale_bytes = 0;
+  if (M.format == MOE_FMT_Q4_AFFINE_G64) {
+    if (!M.scales || !M.biases) return MOE_ERR_NULL_POINTER;
+    if (!aligned(M.scales, 2) || !aligned(M.biases, 2)) return MOE_ERR_MISALIGNED;
+    scale_bytes = (size_t)n * (k / 64) * 2;
+  } else if (M.format == MOE_FMT_NVFP4) {
+    if (!M.scales || !M.tensor_scale) return MOE_ERR_NULL_POINTER;
+    if (!aligned(M.scales, 2) || !aligned(M.tensor_scale, 4)) return MOE_ERR_MISALIGNED;
+    scale_bytes = (size_t)n * (k / 16);
+  }
+  if (scale_bytes && E > 1 && (M.scale_stride < (int64_t)scale_bytes || M.scale_stride % 2))
+    return M.scale_stride % 2 ? MOE_ERR_MISALIGNED : MOE_ERR_BAD_SHAPE;
+  out->packed = (const uint8_t*)M.packed;
+  out->scales = (const uint8_t*)M.scales;
+  out->biases = (const uint8_t*)M.biases;
+  out->tscale = M.tensor_scale;
+  out->estride = E > 1 ? M.expert_stride : (long long)mat_bytes;
+  out->sstride = E > 1 ? M.scale_stride : (long long)scale_bytes;
+  out->fmt = M.format;
+  out->n = n;
+  out->k = k;
+  return MOE_OK;
+}
+
+int check_table(const moe_expert_table* t, int inter, int h, int E, MatDev* g, MatDev* u,
+                MatDev* d) {
+  if (!t) return MOE_ERR_NULL_POINTER;
+  if (t->gate.format != t->up.format) return MOE_ERR_BAD_FORMAT;
+  int rc;
+  if ((rc = check_matrix(t->gate, inter, h, E, g))) return rc;
+  if ((rc = check_matrix(t->up, inter, h, E, u))) return rc;
+  if ((rc = check_matrix(t->down, h, inter, E, d))) return rc;
+  return MOE_OK;
+}
+
+int n_tiles_c_of(int h) { return (h + kColsPerCta - 1) / kColsPerCta; }
+
+WsLayout layout_of(const moe_cfg* c, int m) {
+  return make_layout(m, c->hidden, c->num_experts, c->top_k, c->moe_inter, c->shared_inter,
+                     n_tiles_c_of(c->hidden));
+}
+
+// Compute capability 10.0 check, cached per device.
+int check_device() {
+  static std::mutex mu;
+  static int state[64] = {0};  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (state[dev] == 0) {
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)))
+      return cuda_fail(e);
+    state[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return state[dev] == 1 ? MOE_OK : MOE_ERR_UNSUPPORTED_DEVICE;
+}
+
+// Launch with programmatic stream serialisation (PDL) so a kernel's prologue overlaps the
+// previous kernel's tail; smem > 48 KB is opted into once per kernel.
+template <typename K>
+cudaError_t launch(K kernel, int grid, int block, size_t smem, cudaStream_t st, const Params& p,
+                   bool pdl) {
+  if (smem > 48 * 1024) {
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+// Rows staged per pass: as many (1, 2 or 4) as fit a 80 KB staging budget, never more than m.
+int rows_per_pass(int K, int fmt, int m) {
+  const size_t per_row = (size_t)K * 4 + (fmt == MOE_FMT_Q4_AFFINE_G64 ? (size_t)K / 8 : 0);
+  int rb = 4;
+  while (rb > 1 && per_row * rb > 80 * 1024) rb >>= 1;
+  while (rb > 1 && rb / 2 >= m) rb >>= 1;
+  return rb;
+}
+
+size_t staging_bytes(int K, int fmt, int rb) {
+  return (size_t)rb * K * 4 + (fmt == MOE_FMT_Q4_AFFINE_G64 ? (size_t)rb * (K / 32) * 4 : 0);
+}
+
+template <int FMT, bool XBF16>
+cudaError_t launch_gate_up_fmt(int rb, int grid, size_t smem, cudaStream_t st, const Params& p) {
+  switch (rb) {
+    case 1: return launch(gate_up_swiglu_kernel<FMT, XBF16, 1>, grid, kThreads, smem, st, p, true);
+    case 2: return launch(gate_up_swiglu_kernel<FMT, XBF16, 2>, grid, kThreads, smem, st, p, true);
+    default: return launch(gate_up_swiglu_kernel<FMT, XBF16, 4>, grid, kThreads, smem, st, p, true);
+  }
+}
+
+template <bool XBF16>
+cudaError_t launch_gate_up(int fmt, int rb, int grid, size_t smem, cudaStream_t st,
+                           const Params& p) {
+  switch (fmt) {
+    case MOE_FMT_F32: return launch_gate_up_fmt<MOE_FMT_F32, XBF16>(rb, grid, smem, st, p);
+    case MOE_FMT_BF16: return launch_gate_up_fmt<MOE_FMT_BF16, XBF16>(rb, grid, smem, st, p);
+    case MOE_FMT_Q4_AFFINE_G64:
+      return launch_gate_up_fmt<MOE_FMT_Q4_AFFINE_G64, XBF16>(rb, grid, smem, st, p);
+    default: return launch_gate_up_fmt<MOE_FMT_NVFP4, XBF16>(rb, grid, smem, st, p);
+  }
+}
+
+template <int FMT>
+cudaError_t launch_down_fmt(int rb, int grid, size_t smem, cudaStream_t st, const Params& p) {
+  switch (rb) {
+    case 1: return launch(down_blend_kernel<FMT, 1>, grid, kThreads, smem, st, p, true);
+    case 2: return launch(down_blend_kernel<FMT, 2>, grid, kThreads, smem, st, p, true);
+    default: return launch(down_blend_kernel<FMT, 4>, grid, kThreads, smem, st, p, true);
+  }
+}
+
+cudaError_t launch_down(int fmt, int rb, int grid, size_t smem, cudaStream_t st,
+                        const Params& p) {
+  switch (fmt) {
+    case MOE_FMT_F32: return launch_down_fmt<MOE_FMT_F32>(rb, grid, smem, st, p);
+    case MOE_FMT_BF16: return launch_down_fmt<MOE_FMT_BF16>(rb, grid, smem, st, p);
+    case MOE_FMT_Q4_AFFINE_G64: return launch_down_fmt<MOE_FMT_Q4_AFFINE_G64>(rb, grid, smem, st, p);
+    default: return launch_down_fmt<MOE_FMT_NVFP4>(rb, grid, smem, st, p);
+  }
+}
+
+}  // namespace
+
+extern "C" int moe_workspace_bytes(const moe_cfg* cfg, int m, size_t* out_bytes) {
+  if (!out_bytes) return MOE_ERR_NULL_POINTER;
+  const int rc = check_cfg(cfg, m);
+  if (rc) return rc;
+  *out_bytes = layout_of(cfg, m).total;
+  return MOE_OK;
+}
+
+extern "C" int moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace) return MOE_ERR_NULL_POINTER;
+  if (workspace_bytes < (size_t)kCtrlBytes) return MOE_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return MOE_ERR_MISALIGNED;
+  const cudaError_t e = cudaMemsetAsync(workspace, 0, kCtrlBytes, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, const void* router_w,
+                                  const float* expert_bias, const moe_expert_table* routed,
+                                  const moe_expert_table* shared, const void* shared_gate_w,
+                                  void* out, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  int rc = check_cfg(cfg, m);
+  if (rc) return rc;
+  const moe_cfg& c = *cfg;
+  if (!x || !router_w || !routed || !out || !workspace) return MOE_ERR_NULL_POINTER;
+  if (!aligned(x, 16) || !aligned(router_w, 16) || !aligned(out, 16) || !aligned(workspace, 256))
+    return MOE_ERR_MISALIGNED;
+  if (c.has_expert_bias && !expert_bias) return MOE_ERR_NULL_POINTER;
+  if (expert_bias && !aligned(expert_bias, 4)) return MOE_ERR_MISALIGNED;
+  const bool has_shared = c.shared_kind != MOE_SHARED_NONE;
+  if (has_shared && !shared) return MOE_ERR_NULL_POINTER;
+  if (c.shared_kind == MOE_SHARED_SIGMOID_GATE) {
+    if (!shared_gate_w) return MOE_ERR_NULL_POINTER;
+    if (!aligned(shared_gate_w, 16)) return MOE_ERR_MISALIGNED;
+  }
+  Params p;
+  std::memset(&p, 0, sizeof(p));
+  if ((rc = check_table(routed, c.moe_inter, c.hidden, c.num_experts, &p.rg, &p.ru, &p.rd)))
+    return rc;
+  if (has_shared &&
+      (rc = check_table(shared, c.shared_inter, c.hidden, 1, &p.sg, &p.su, &p.sd)))
+    return rc;
+  const WsLayout L = layout_of(&c, m);
+  if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if ((rc = check_device())) return rc;
+
+  p.m = m;
+  p.h = c.hidden;
+  p.E = c.num_experts;
+  p.k = c.top_k;
+  p.I = c.moe_inter;
+  p.S = has_shared ? c.shared_inter : 0;
+  p.routing = c.routing;
+  p.norm = c.norm_topk_prob;
+  p.raw = c.select_on_raw_logits;
+  p.has_bias = c.has_expert_bias;
+  p.before_ffn = c.weight_before_ffn;
+  p.shared_kind = c.shared_kind;
+  p.out_bf16 = c.out_dtype == MOE_FMT_BF16;
+  p.rsf = c.routed_scaling_factor;
+  const int te = m * c.top_k;
+  p.cap = te < c.num_experts ? te : c.num_experts;
+  p.n_tiles_i = (c.moe_inter + kRowsPerCta - 1) / kRowsPerCta;
+  p.n_tiles_s = has_shared ? (p.S + kRowsPerCta - 1) / kRowsPerCta : 0;
+  p.n_tiles_c = n_tiles_c_of(c.hidden);
+  p.has_shared = has_shared ? 1 : 0;
+  p.x = x;
+  p.router_w = router_w;
+  p.expert_bias = expert_bias;
+  p.shared_gate_w = shared_gate_w;
+  p.out = out;
+  uint8_t* ws = (uint8_t*)workspace;
+  p.ctrl = (unsigned*)ws;
+  p.logits = (float*)(ws + L.logits);
+  p.idx = (int*)(ws + L.idx);
+  p.wts = (float*)(ws + L.wts);
+  p.gamma = (float*)(ws + L.gamma);
+  p.sorted_pairs = (int*)(ws + L.sorted_pairs);
+  p.offsets = (int*)(ws + L.offsets);
+  p.token_to_perm = (int*)(ws + L.token_to_perm);
+  p.active = (int*)(ws + L.active);
+  p.active_count = (int*)(ws + L.active_count);
+  p.act = (float*)(ws + L.act);
+  p.act_sh = (float*)(ws + L.act_sh);
+  p.ypart = (float*)(ws + L.ypart);
+  p.ysh = (float*)(ws + L.ysh);
+  p.tickets = (unsigned*)(ws + L.tickets);
+
+  cudaStream_t st = (cudaStream_t)stream;
+  const bool xbf16 = c.x_dtype == MOE_FMT_BF16;
+  const int router_grid = c.num_experts + (c.shared_kind == MOE_SHARED_SIGMOID_GATE ? 1 : 0);
+  cudaError_t e = xbf16 ? launch(router_topk_group_kernel<true>, router_grid, kRouterThreads, 0,
+                                 st, p, false)
+                        : launch(router_topk_group_kernel<false>, router_grid, kRouterThreads, 0,
+                                 st, p, false);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  // gate + up + SwiGLU: shared tiles first (they need no routing), then routed tiles; one
+  // launch when routed and shared experts share a format, else one launch per format.
+  const int fmt_gu = routed->gate.format;
+  const bool split_gu = has_shared && shared->gate.format != fmt_gu;
+  auto gate_up = [&](int fmt, const Params& q, int grid) {
+    const int rb = rows_per_pass(c.hidden, fmt, m);
+    const size_t smem = staging_bytes(c.hidden, fmt, rb);
+    return xbf16 ? launch_gate_up<true>(fmt, rb, grid, smem, st, q)
+                 : launch_gate_up<false>(fmt, rb, grid, smem, st, q);
+  };
+  if (split_gu) {
+    Params ps = p;  // shared tiles only
+    e = gate_up(shared->gate.format, ps, p.n_tiles_s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    Params pr = p;  // routed tiles only
+    pr.n_tiles_s = 0;
+    e = gate_up(fmt_gu, pr, p.cap * p.n_tiles_i);
+  } else {
+    e = gate_up(fmt_gu, p, p.n_tiles_s + p.cap * p.n_tiles_i);
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  // down + blend. The column-tile tickets count routed and shared arrivals across launches, so
+  // a shared expert in another format runs as a second launch (its CTAs arrive last).
+  const int fmt_d = routed->down.format;
+  const bool split_d = has_shared && shared->down.format != fmt_d;
+  auto down = [&](int fmt, const Params& q, int grid, int K) {
+    const int rb = rows_per_pass(K, fmt, m);
+    return launch_down(fmt, rb, grid, staging_bytes(K, fmt, rb), st, q);
+  };
+  if (split_d) {
+    e = down(fmt_d, p, p.n_tiles_c * p.cap, c.moe_inter);
+    if (e != cudaSuccess) return cuda_fail(e);
+    Params ps = p;
+    ps.slot_base = p.cap;
+    e = down(shared->down.format, ps, p.n_tiles_c, p.S);
+  } else {
+    const int kmax = (has_shared && p.S > c.moe_inter) ? p.S : c.moe_inter;
+    e = down(fmt_d, p, p.n_tiles_c * (p.cap + p.has_shared), kmax);
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  return MOE_OK;
+}
+
+extern "C" int moe_decode_read_routing(const moe_cfg* cfg, int m, const void* workspace,
+                                       size_t workspace_bytes, void* stream, int32_t* idx,
+                                       float* weights, int32_t* sorted_pairs,
+                                       int32_t* expert_offsets, int32_t* token_to_perm,
+                                       int32_t* active, int32_t* active_count, float* gamma) {
+  int rc = check_cfg(cfg, m);
+  if (rc) return rc;
+  if (!workspace) return MOE_ERR_NULL_POINTER;
+  const WsLayout L = layout_of(cfg, m);
+  if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+  const uint8_t* ws = (const uint8_t*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t te = (size_t)m * cfg->top_k;
+  const size_t cap = te < (size_t)cfg->num_experts ? te : (size_t)cfg->num_experts;
+  struct Item { void* dst; size_t off, bytes; } items[] = {
+      {idx, L.idx, te * 4},
+      {weights, L.wts, te * 4},
+      {sorted_pairs, L.sorted_pairs, te * 4},
+      {expert_offsets, L.offsets, (size_t)(cfg->num_experts + 1) * 4},
+      {token_to_perm, L.token_to_perm, te * 4},
+      {active, L.active, cap * 4},
+      {active_count, L.active_count, 4},
+      {gamma, L.gamma, (size_t)m * 4},
+  };
+  for (const Item& it : items) {
+    if (!it.dst) continue;
+    const cudaError_t e = cudaMemcpyAsync(it.dst, ws + it.off, it.bytes, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  const cudaError_t e = cudaStreamSynchronize(st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+extern "C" int moe_get_device_status(const void* workspace, size_t workspace_bytes, void* stream,
+                                     int32_t* status) {
+  if (!workspace || !status) return MOE_ERR_NULL_POINTER;
+  if (workspace_bytes < (size_t)kCtrlBytes) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(status, workspace, 4, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+}
+
+extern "C" const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case MOE_ERR_BAD_SHAPE: return "invalid shape (m, hidden, experts, top_k or intermediate)";
+    case MOE_ERR_BAD_FORMAT: return "invalid or mismatched format";
+    case MOE_ERR_BAD_OPTION: return "invalid routing or shared-expert option";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_MISALIGNED: return "pointer or stride misaligned";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_UNSUPPORTED_DEVICE: return "device is not compute capability 10.0 (B200)";
+    case MOE_ERR_DEVICE_CHECK: return "device-side consistency check failed";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+extern "C" int moe_version(void) { return 100; }

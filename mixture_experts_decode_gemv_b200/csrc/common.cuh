@@ -1,0 +1,129 @@
+// Shared definitions of the decode MoE kernels: launch parameters, workspace layout, small PTX
+// helpers. Device code targets sm_100a only.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "../../include/moe_decode.h"
+
+namespace moe {
+
+// Work-tile geometry shared by the host launcher and the kernels.
+constexpr int kThreads = 256;          // 8 warps per CTA in the expert kernels
+constexpr int kWarps = kThreads / 32;
+constexpr int kLanesPerRow = 8;        // one weight row per 8 lanes, 16 bytes per lane per step
+constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+constexpr int kRowsPerCta = kWarps * kRowsPerWarp;  // 32 gate/up row pairs per CTA tile
+constexpr int kColsPerCta = 2 * kRowsPerCta;       // 64 down-projection output columns per CTA
+constexpr int kRouterThreads = 128;
+constexpr int kCtrlBytes = 256;
+
+// Control words at the start of the workspace.
+enum CtrlWord { kStatus = 0, kRouterTicket = 1 };
+
+struct MatDev {
+  const uint8_t* packed;
+  const uint8_t* scales;
+  const uint8_t* biases;
+  const float* tscale;
+  long long estride;   // bytes between experts (packed)
+  long long sstride;   // bytes between experts (scales / biases)
+  int fmt;
+  int n, k;            // rows and columns of one expert matrix
+};
+
+// Byte offsets of the workspace regions (all 256-byte aligned).
+struct WsLayout {
+  size_t logits, idx, wts, gamma, sorted_pairs, offsets, token_to_perm, active, active_count;
+  size_t act, act_sh, ypart, ysh, tickets, total;
+};
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+inline WsLayout make_layout(int m, int h, int E, int k, int I, int S, int n_tiles_c) {
+  WsLayout L;
+  const size_t te = (size_t)m * k;
+  const size_t cap = te < (size_t)E ? te : (size_t)E;
+  size_t off = kCtrlBytes;
+  auto take = [&](size_t bytes) { size_t at = off; off = align256(off + bytes); return at; };
+  L.logits = take((size_t)m * (E + 1) * 4);
+  L.idx = take(te * 4);
+  L.wts = take(te * 4);
+  L.gamma = take((size_t)m * 4);
+  L.sorted_pairs = take(te * 4);
+  L.offsets = take((size_t)(E + 1) * 4);
+  L.token_to_perm = take(te * 4);
+  L.active = take(cap * 4);
+  L.active_count = take(4);
+  L.act = take(te * (size_t)I * 4);
+  L.act_sh = take((size_t)m * (S > 0 ? S : 1) * 4);
+  L.ypart = take(te * (size_t)h * 4);
+  L.ysh = take((size_t)m * h * 4);
+  L.tickets = take((size_t)n_tiles_c * 4);
+  L.total = off;
+  return L;
+}
+
+struct Params {
+  int m, h, E, k, I, S;
+  int routing, norm, raw, has_bias, before_ffn, shared_kind, out_bf16;
+  float rsf;
+  int cap;             // min(m*k, E): routed work slots
+  int n_tiles_i;       // routed gate/up tiles per expert
+  int n_tiles_s;       // shared gate/up tiles
+  int n_tiles_c;       // output-column tiles of the down projection
+  int has_shared;
+  int slot_base;       // first work slot of a down launch (shared-only launches start at cap)
+  const void* x;
+  const void* router_w;
+  const float* expert_bias;
+  const void* shared_gate_w;
+  MatDev rg, ru, rd;   // routed gate, up, down
+  MatDev sg, su, sd;   // shared gate, up, down
+  void* out;
+  unsigned* ctrl;
+  float* logits;
+  int* idx;
+  float* wts;
+  float* gamma;
+  int* sorted_pairs;
+  int* offsets;
+  int* token_to_perm;
+  int* active;
+  int* active_count;
+  float* act;
+  float* act_sh;
+  float* ypart;
+  float* ysh;
+  unsigned* tickets;
+};
+
+// ---- PTX helpers -------------------------------------------------------------------------------
+
+// Streaming 16-byte load of weights: read-only path, no L1 allocation.
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// Programmatic dependent launch: wait for the preceding grid's completion (no-op without PDL)
+// and allow the next grid to start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + __expf(-z)); }
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+}  // namespace moe

@@ -1,0 +1,264 @@
+// Router GEMV, top-k routing and grouping of (row, slot) pairs by expert, in one launch.
+//
+// Every CTA computes the logits of one router row (one expert, or the shared-expert gate vector)
+// for all m activation rows. The CTA that finishes last (an atomic ticket, no spinning) then
+// routes every row and groups the pairs by expert:
+//   - routing per row follows the options of the layer (softmax, or sigmoid with an optional
+//     expert bias for selection only, raw-logit selection, norm_topk_prob, routed scaling);
+//   - grouping is a stable counting sort of pair ids p = r*k + s by expert id, giving
+//     sorted_pairs, expert_offsets, token_to_perm, the ascending active-expert list and its count
+//     (the sort step of metrale "forward_bf16_grouped_decode.rs").
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+template <bool XBF16>
+__device__ __forceinline__ float dot_chunk16(uint4 w, uint4 x) {
+  if constexpr (XBF16) {
+    float a = bf16lo(w.x) * bf16lo(x.x);
+    a = fmaf(bf16hi(w.x), bf16hi(x.x), a);
+    a = fmaf(bf16lo(w.y), bf16lo(x.y), a);
+    a = fmaf(bf16hi(w.y), bf16hi(x.y), a);
+    a = fmaf(bf16lo(w.z), bf16lo(x.z), a);
+    a = fmaf(bf16hi(w.z), bf16hi(x.z), a);
+    a = fmaf(bf16lo(w.w), bf16lo(x.w), a);
+    a = fmaf(bf16hi(w.w), bf16hi(x.w), a);
+    return a;
+  } else {
+    float a = __uint_as_float(w.x) * __uint_as_float(x.x);
+    a = fmaf(__uint_as_float(w.y), __uint_as_float(x.y), a);
+    a = fmaf(__uint_as_float(w.z), __uint_as_float(x.z), a);
+    a = fmaf(__uint_as_float(w.w), __uint_as_float(x.w), a);
+    return a;
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Routing of row r by one warp: selection keys, k rounds of warp arg-max (ties to the lower
+// id), weights. Writes idx / wts (global) and s_idx (shared).
+__device__ void route_row_warp(const Params& p, int r, int* s_idx) {
+  const int lane = threadIdx.x & 31;
+  const int E = p.E, k = p.k;
+  const float* lrow = p.logits + (size_t)r * (E + 1);
+  float lg[8], key[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane + 32 * j;
+    const bool valid = e < E;
+    const float l = valid ? __ldcg(lrow + e) : -INFINITY;
+    lg[j] = l;
+    float kv = l;
+    if (p.routing == MOE_ROUTE_SIGMOID && !p.raw) {
+      kv = 1.0f / (1.0f + expf(-l));
+      if (p.has_bias && valid) kv += __ldg(p.expert_bias + e);
+    }
+    key[j] = valid ? kv : -INFINITY;
+  }
+  float mx = -INFINITY, den = 0.f;
+  if (p.routing == MOE_ROUTE_SOFTMAX) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mx = fmaxf(mx, lg[j]);
+    mx = warp_max(mx);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) den += (lane + 32 * j < E) ? expf(lg[j] - mx) : 0.f;
+    den = warp_sum(den);
+  }
+  unsigned taken = 0;
+  int my_id = 0;
+  float my_l = 0.f;
+  bool bad = false;
+  for (int s = 0; s < k; ++s) {
+    float bk = -INFINITY;
+    int bid = 0x7fffffff;
+    float bl = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && !((taken >> j) & 1u) && (key[j] > bk || (key[j] == bk && e < bid))) {
+        bk = key[j];
+        bid = e;
+        bl = lg[j];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+      const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
+      if (ok > bk || (ok == bk && oid < bid)) {
+        bk = ok;
+        bid = oid;
+        bl = ol;
+      }
+    }
+    if (bid >= E) {  // only NaN keys left: keep every index in range and flag the row
+      bad = true;
+      bid = s;
+    }
+    if ((bid & 31) == lane) taken |= 1u << (bid >> 5);
+    if (lane == s) {
+      my_id = bid;
+      my_l = bl;
+    }
+  }
+  float wv = 0.f;
+  if (lane < k) {
+    wv = (p.routing == MOE_ROUTE_SOFTMAX) ? expf(my_l - mx) / den : 1.0f / (1.0f + expf(-my_l));
+  }
+  if (p.norm) {
+    const float tot = warp_sum(lane < k ? wv : 0.f);
+    wv = wv / tot;
+  }
+  wv *= p.rsf;
+  if (lane < k) {
+    p.idx[r * k + lane] = my_id;
+    p.wts[r * k + lane] = wv;
+    s_idx[r * k + lane] = my_id;
+  }
+  if (lane == 0) {
+    if (p.shared_kind == MOE_SHARED_SIGMOID_GATE) {
+      p.gamma[r] = 1.0f / (1.0f + expf(-__ldcg(lrow + E)));
+    }
+    if (bad) atomicExch(p.ctrl + kStatus, (unsigned)MOE_ERR_DEVICE_CHECK);
+  }
+}
+
+// Stable counting sort of the te pairs by expert (run by one CTA of kRouterThreads threads).
+__device__ void group_pairs(const Params& p, const int* s_idx) {
+  __shared__ int s_cnt[MOE_MAX_EXPERTS];
+  __shared__ int s_off[MOE_MAX_EXPERTS + 1];
+  __shared__ int s_wsum[kRouterThreads / 32][2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = p.E, te = p.m * p.k;
+  for (int e = tid; e < MOE_MAX_EXPERTS; e += kRouterThreads) s_cnt[e] = 0;
+  __syncthreads();
+  for (int q = tid; q < te; q += kRouterThreads) atomicAdd(&s_cnt[s_idx[q]], 1);
+  __syncthreads();
+  // exclusive scan of counts and of the non-empty flags; thread t owns experts 2t, 2t+1
+  const int e0 = 2 * tid, e1 = 2 * tid + 1;
+  const int c0 = e0 < E ? s_cnt[e0] : 0, c1 = e1 < E ? s_cnt[e1] : 0;
+  const int f0 = c0 > 0, f1 = c1 > 0;
+  int cs = c0 + c1, fs = f0 + f1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, cs, o), b = __shfl_up_sync(0xffffffffu, fs, o);
+    if (lane >= o) {
+      cs += a;
+      fs += b;
+    }
+  }
+  if (lane == 31) {
+    s_wsum[warp][0] = cs;
+    s_wsum[warp][1] = fs;
+  }
+  __syncthreads();
+  int cbase = 0, fbase = 0;
+  for (int w = 0; w < warp; ++w) {
+    cbase += s_wsum[w][0];
+    fbase += s_wsum[w][1];
+  }
+  const int cexcl = cbase + cs - (c0 + c1), fexcl = fbase + fs - (f0 + f1);
+  if (e0 < E) {
+    s_off[e0] = cexcl;
+    p.offsets[e0] = cexcl;
+    if (f0) p.active[fexcl] = e0;
+  }
+  if (e1 < E) {
+    s_off[e1] = cexcl + c0;
+    p.offsets[e1] = cexcl + c0;
+    if (f1) p.active[fexcl + f0] = e1;
+  }
+  if (tid == kRouterThreads - 1) {
+    p.offsets[E] = te;
+    *p.active_count = fbase + fs;
+  }
+  __syncthreads();
+  for (int q = tid; q < te; q += kRouterThreads) {
+    const int e = s_idx[q];
+    int rank = 0;
+    for (int q2 = 0; q2 < q; ++q2) rank += (s_idx[q2] == e);
+    const int pos = s_off[e] + rank;
+    p.sorted_pairs[pos] = q;
+    p.token_to_perm[q] = pos;
+  }
+}
+
+template <bool XBF16>
+__global__ void __launch_bounds__(kRouterThreads) router_topk_group_kernel(
+    const __grid_constant__ Params p) {
+  pdl_launch_dependents();
+  const int erow = blockIdx.x;  // router row; erow == E is the shared-expert gate vector
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int esz = XBF16 ? 2 : 4;
+  const size_t row_bytes = (size_t)p.h * esz;
+  const int nch = (int)(row_bytes / 16);
+  const uint8_t* wrow = erow < p.E ? (const uint8_t*)p.router_w + (size_t)erow * row_bytes
+                                   : (const uint8_t*)p.shared_gate_w;
+  const uint8_t* xb = (const uint8_t*)p.x;
+  __shared__ float s_red[kRouterThreads / 32][8];
+  __shared__ int s_last;
+  __shared__ int s_idx[MOE_MAX_ROWS * MOE_MAX_TOP_K];
+
+  for (int rb = 0; rb < p.m; rb += 8) {
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    for (int c = tid; c < nch; c += kRouterThreads) {
+      const uint4 w = ldg_stream(wrow + (size_t)c * 16);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (rb + j < p.m) {
+          const uint4 xv = __ldg((const uint4*)(xb + (size_t)(rb + j) * row_bytes) + c);
+          acc[j] += dot_chunk16<XBF16>(w, xv);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float v = warp_sum(acc[j]);
+      if (lane == 0) s_red[warp][j] = v;
+    }
+    __syncthreads();
+    if (tid < 8 && rb + tid < p.m) {
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kRouterThreads / 32; ++w) v += s_red[w][tid];
+      p.logits[(size_t)(rb + tid) * (p.E + 1) + erow] = v;
+    }
+    __syncthreads();
+  }
+
+  if (tid == 0) {
+    __threadfence();
+    const unsigned t = atomicAdd(p.ctrl + kRouterTicket, 1u);
+    s_last = (t == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  for (int r = warp; r < p.m; r += kRouterThreads / 32) route_row_warp(p, r, s_idx);
+  __syncthreads();
+  group_pairs(p, s_idx);
+  for (int t = tid; t < p.n_tiles_c; t += kRouterThreads) p.tickets[t] = 0u;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    p.ctrl[kRouterTicket] = 0u;
+  }
+}
+
+}  // namespace moe
