@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--replicas", type=int, default=None,
+                    help="weight replicas (default: enough for 4x L2 between reuses)")
     return ap.parse_args()
 
 
@@ -249,11 +251,12 @@ def run_ours(args, cfg):
     free, _ = torch.cuda.mem_get_info(dev_index)
     r_need = int(math.ceil(4 * l2 / max(1.0, min(bytes_per_batch)))) + 1
     r_cap = max(2, int(0.6 * free // max(1, layer_bytes)))
-    R = max(2, min(r_need, r_cap))
+    R = max(2, min(r_need, r_cap)) if args.replicas is None else max(1, args.replicas)
     reps = [dev0] + [dev0.replica() for _ in range(R - 1)]
 
     G = R * max(1, int(math.ceil(args.graph_len / R)))
-    steps = args.steps if args.steps is not None else max(G, int(2.0e6 / max(1.0, mean_bytes / 6e3)))
+    est_us = mean_bytes / 6.0e6 + 5.0            # ~6 TB/s plus fixed latency, for sizing only
+    steps = args.steps if args.steps is not None else max(G, int(2.0e6 / est_us))
     steps = max(1, steps)
 
     def seq(n, start=0):
@@ -285,12 +288,13 @@ def run_ours(args, cfg):
     torch.cuda.synchronize()
     clocks = ClockSampler(dev_index, enabled=not args.no_clocks)
     time.sleep(0.3)
-    start.record(stream)
-    for _ in range(n_full):
-        g_full.replay()
-    if g_rem is not None:
-        g_rem.replay()
-    end.record(stream)
+    with torch.cuda.stream(stream):  # graphs replay on the current stream: keep it `stream`
+        start.record(stream)
+        for _ in range(n_full):
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        end.record(stream)
     torch.cuda.synchronize()
     barrier(wsz)
     clk = clocks.stop()
@@ -325,7 +329,7 @@ def run_ours(args, cfg):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), wsz)
 
-    kernels_per_step = 3 + (1 if cfg.has_shared and False else 0)
+    kernels_per_step = 3
     result = {
         "metric": METRIC,
         "value": wsz * m * steps / (ms * 1e-3),

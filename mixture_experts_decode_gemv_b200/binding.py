@@ -188,6 +188,7 @@ def moe_decode_read_routing(cfg: moe_cfg, m: int, workspace, workspace_bytes: in
                                        "token_to_perm", "active", "active_count", "gamma")])
     _check(rc, "moe_decode_read_routing")
     out["active_count"] = int(out["active_count"][0])
+    out["active"] = out["active"][: max(0, min(cap, out["active_count"]))]
     out["idx"] = out["idx"].reshape(m, cfg.top_k)
     out["w"] = out["w"].reshape(m, cfg.top_k)
     return out
