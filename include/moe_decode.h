@@ -176,6 +176,33 @@ int moe_get_device_status(const void* workspace, size_t workspace_bytes, void* s
                           int32_t* status);
 
 /* ------------------------------------------------------------------------------------------ */
+/* The layer without a caller workspace                                                        */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Not from the pages this library follows (they have no counterpart): an addition for callers
+ * that cannot give the library device memory. Typical ones are plugins hosted by an inference
+ * server or graph runtime whose op interface passes only the op's own tensors and which must not
+ * call cudaMalloc/cudaFree while serving (those calls synchronise the device and can fail under
+ * memory pressure), and programs that reserve all of their device memory at start-up.
+ *
+ * Same arguments and results as moe_decode_forward, without the workspace. The scratch is one
+ * fixed array of MOE_NO_ALLOC_SCRATCH_BYTES in the library's device image; every GPU that loads
+ * the library keeps it until the process exits. A call whose moe_workspace_bytes(cfg, m) exceeds
+ * that size is refused with MOE_ERR_WORKSPACE, and any other bad argument with the error
+ * moe_decode_forward gives; a refused call launches nothing. The first call on a device looks up
+ * the array's device address (cudaGetSymbolAddress, with that device current): make that first
+ * call before any stream capture. Every call then clears the array's control words
+ * (cudaMemsetAsync on `stream`) and runs the layer; it allocates nothing.
+ * All calls on a device share the one array, which keeps the last call's contents: calls that
+ * overlap on the GPU (other streams, or host threads whose calls are not ordered) race on it and
+ * corrupt each other's results. Routing read-back and device status are not available for it. */
+#define MOE_NO_ALLOC_SCRATCH_BYTES (16u << 20)
+int moe_decode_forward_no_alloc(const moe_cfg* cfg, int m, const void* x, const void* router_w,
+                                const float* expert_bias, const moe_expert_table* routed,
+                                const moe_expert_table* shared, const void* shared_gate_w,
+                                void* out, void* stream);
+
+/* ------------------------------------------------------------------------------------------ */
 /* Pack and quantise helpers (host memory only, synchronous, no GPU needed)                     */
 /* ------------------------------------------------------------------------------------------ */
 

@@ -47,8 +47,10 @@ EXPORTS = (
     "moe_workspace_bytes", "moe_workspace_init", "moe_decode_forward", "moe_decode_read_routing",
     "moe_get_device_status", "moe_packed_bytes", "moe_pack_bf16", "moe_quantize_q4_affine",
     "moe_quantize_nvfp4", "moe_dequantize", "moe_status_string", "moe_last_cuda_error",
-    "moe_version",
+    "moe_version", "moe_decode_forward_no_alloc",
 )
+
+MOE_NO_ALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class MoeError(RuntimeError):
@@ -105,6 +107,8 @@ def _load() -> ctypes.CDLL:
         "moe_quantize_q4_affine": [vp, i32, i32, vp, vp, vp],
         "moe_quantize_nvfp4": [vp, i32, i32, vp, vp, vp],
         "moe_dequantize": [i32, vp, vp, vp, vp, i32, i32, vp],
+        "moe_decode_forward_no_alloc": [P(moe_cfg), i32, vp, vp, vp, P(moe_expert_table),
+                                        P(moe_expert_table), vp, vp, vp],
         "moe_status_string": [i32],
         "moe_last_cuda_error": [],
         "moe_version": [],
@@ -169,6 +173,17 @@ def moe_decode_forward(cfg: moe_cfg, m: int, x, router_w, expert_bias, routed: m
         ctypes.byref(shared) if shared is not None else None, _ptr(shared_gate_w), _ptr(out),
         _ptr(workspace), workspace_bytes, _stream(stream))
     _check(rc, "moe_decode_forward")
+
+
+def moe_decode_forward_no_alloc(cfg: moe_cfg, m: int, x, router_w, expert_bias,
+                                routed: moe_expert_table, shared: Optional[moe_expert_table],
+                                shared_gate_w, out, stream=None) -> None:
+    """The layer with the library's fixed device scratch instead of a caller workspace."""
+    rc = lib.moe_decode_forward_no_alloc(
+        ctypes.byref(cfg), m, _ptr(x), _ptr(router_w), _ptr(expert_bias), ctypes.byref(routed),
+        ctypes.byref(shared) if shared is not None else None, _ptr(shared_gate_w), _ptr(out),
+        _stream(stream))
+    _check(rc, "moe_decode_forward_no_alloc")
 
 
 def moe_decode_read_routing(cfg: moe_cfg, m: int, workspace, workspace_bytes: int, stream=None):

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoedecode.so")
 
-SOURCES = ["api.cu", "host_formats.cpp"]
+SOURCES = ["api.cu", "host_formats.cpp", "no_alloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
