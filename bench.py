@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--path", choices=("auto", "chain"), default="auto",
+                    help="launch path: automatic (persistent kernel for m <= 4) or the chain")
     ap.add_argument("--replicas", type=int, default=None,
                     help="weight replicas (default: enough for 4x L2 between reuses)")
     return ap.parse_args()
@@ -381,6 +383,8 @@ def main():
     args = parse_args()
     from mixture_experts_decode_gemv_b200.synthetic import CONFIGS
     cfg = CONFIGS[args.config]
+    if args.path == "chain":
+        os.environ["MOE_DECODE_PATH"] = "chain"
     if args.m < 1 or args.m > 64:
         raise SystemExit("--m must be in 1..64")
     if args.impl == "reference":

@@ -8,8 +8,11 @@
 #include <cstring>
 #include <mutex>
 
+#include <cstdlib>
+
 #include "common.cuh"
 #include "experts.cuh"
+#include "fused.cuh"
 #include "router.cuh"
 
 using namespace moe;
@@ -210,6 +213,115 @@ cudaError_t launch_down(int fmt, int rb, int grid, size_t smem, cudaStream_t st,
   }
 }
 
+// ---- persistent single-kernel path (m <= 4) --------------------------------------------------
+
+int sm_count() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) cudaDeviceGetAttribute(&cache[dev], cudaDevAttrMultiProcessorCount, dev);
+  return cache[dev];
+}
+
+// Debug / test knob, read on every call: MOE_DECODE_PATH=chain forces the three-kernel chain
+// (default: automatic choice).
+int forced_path() {
+  const char* e = std::getenv("MOE_DECODE_PATH");
+  return (e && !std::strcmp(e, "chain")) ? 1 : 0;
+}
+
+size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
+constexpr size_t kFusedSmemBudget = 220 * 1024;
+
+// Shared-memory plan of the persistent kernel; false when the layer does not fit it.
+bool plan_fused(const moe_cfg& c, int m, bool has_shared, int fmt, int sms, FusedPlan* fp) {
+  if (m > kFusedMaxRows || sms <= 0) return false;
+  const int te = m * c.top_k, n_rows = te + (has_shared ? m : 0);
+  const int kmax = (has_shared && c.shared_inter > c.moe_inter) ? c.shared_inter : c.moe_inter;
+  const int ld = (kmax + 31) / 32 * 32;
+  const int cols = (c.hidden + sms - 1) / sms;
+  const bool q4 = fmt == MOE_FMT_Q4_AFFINE_G64;
+  size_t off = 0;
+  fp->xs_off = (int)off;
+  off += align16((size_t)m * c.hidden * 4);
+  fp->xsum_off = (int)off;
+  off += q4 ? align16((size_t)m * (c.hidden / 32) * 4) : 0;
+  fp->act_off = (int)off;
+  off += align16((size_t)n_rows * ld * 4);
+  fp->actsum_off = (int)off;
+  off += q4 ? align16((size_t)n_rows * (ld / 32) * 4) : 0;
+  fp->y_off = (int)off;
+  off += align16((size_t)n_rows * cols * 4);
+  if (off > kFusedSmemBudget) return false;
+  fp->grid = sms;
+  fp->cols_per_cta = cols;
+  fp->act_ld = ld;
+  fp->smem_bytes = (int)off;
+  fp->spin_limit = 2000000000LL;  // about a second of clock cycles
+  return true;
+}
+
+template <int FMT, bool XBF16, int RB>
+cudaError_t launch_fused_t(const Params& p, const FusedPlan& fp, cudaStream_t st) {
+  auto kernel = moe_fused_kernel<FMT, FMT, XBF16, RB>;
+  static bool attr_done = false;
+  {
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_done) {
+      const cudaError_t e = cudaFuncSetAttribute(
+          kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedSmemBudget);
+      if (e != cudaSuccess) return e;
+      attr_done = true;
+    }
+  }
+  // every CTA must be resident at once: one CTA per SM, checked for this shared-memory size
+  int per_sm = 0;
+  cudaError_t oe = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kFusedThreads,
+                                                                 fp.smem_bytes);
+  if (oe != cudaSuccess) return oe;
+  if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(fp.grid);
+  cfg.blockDim = dim3(kFusedThreads);
+  cfg.dynamicSmemBytes = fp.smem_bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, p, fp);
+}
+
+template <int FMT, bool XBF16>
+cudaError_t launch_fused_rb(int m, const Params& p, const FusedPlan& fp, cudaStream_t st) {
+  if (m == 1) return launch_fused_t<FMT, XBF16, 1>(p, fp, st);
+  if (m == 2) return launch_fused_t<FMT, XBF16, 2>(p, fp, st);
+  return launch_fused_t<FMT, XBF16, 4>(p, fp, st);
+}
+
+// Formats with a persistent-kernel instantiation (one format for every projection).
+bool fused_formats_ok(int fmt, bool xbf16) {
+  return (fmt == MOE_FMT_F32 && !xbf16) || (xbf16 && (fmt == MOE_FMT_BF16 ||
+                                                      fmt == MOE_FMT_Q4_AFFINE_G64 ||
+                                                      fmt == MOE_FMT_NVFP4));
+}
+
+cudaError_t launch_fused(int fmt, bool xbf16, int m, const Params& p, const FusedPlan& fp,
+                         cudaStream_t st) {
+  switch (fmt) {
+    case MOE_FMT_F32: return launch_fused_rb<MOE_FMT_F32, false>(m, p, fp, st);
+    case MOE_FMT_BF16: return launch_fused_rb<MOE_FMT_BF16, true>(m, p, fp, st);
+    case MOE_FMT_Q4_AFFINE_G64: return launch_fused_rb<MOE_FMT_Q4_AFFINE_G64, true>(m, p, fp, st);
+    default: return launch_fused_rb<MOE_FMT_NVFP4, true>(m, p, fp, st);
+  }
+}
+
 }  // namespace
 
 extern "C" int moe_workspace_bytes(const moe_cfg* cfg, int m, size_t* out_bytes) {
@@ -302,6 +414,22 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
 
   cudaStream_t st = (cudaStream_t)stream;
   const bool xbf16 = c.x_dtype == MOE_FMT_BF16;
+
+  // Host dispatch: one persistent kernel for decode-sized calls when every projection shares a
+  // format and the call's activations fit in shared memory; the three-kernel chain otherwise.
+  {
+    const int fmt = routed->gate.format;
+    const bool one_fmt = routed->down.format == fmt &&
+                         (!has_shared || (shared->gate.format == fmt && shared->down.format == fmt));
+    FusedPlan fp;
+    const int force = forced_path();
+    if (force != 1 && one_fmt && fused_formats_ok(fmt, xbf16) &&
+        plan_fused(c, m, has_shared, fmt, sm_count(), &fp)) {
+      const cudaError_t e = launch_fused(fmt, xbf16, m, p, fp, st);
+      return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+    }
+  }
+
   const int router_grid = c.num_experts + (c.shared_kind == MOE_SHARED_SIGMOID_GATE ? 1 : 0);
   cudaError_t e = xbf16 ? launch(router_topk_group_kernel<true>, router_grid, kRouterThreads, 0,
                                  st, p, false)

@@ -11,6 +11,9 @@
 //   column tile last (atomic ticket, no spinning) blends the tile for every row: the routed slots
 //   in slot order, each times its weight, then gamma times the shared expert.
 // Accumulation is fp32 throughout; activations stay fp32 between the two kernels.
+// The 8-lane reductions are full-warp shuffles, so every guard around them must be uniform
+// across a warp: rows come 4 per warp and I, S (multiples of 4) and h (multiple of 8) keep the
+// `i < N` / `col0 < h` guards warp-uniform (the host refuses other shapes).
 #pragma once
 
 #include <cuda_fp4.h>
@@ -170,7 +173,7 @@ __device__ __forceinline__ void stage_rows(float* xs, float* xsum, int K, int nb
     const uint8_t* g = src(j);
     float* dst = xs + (size_t)j * K;
     if constexpr (SRC_BF16) {
-      for (int c = tid; c < K / 8; c += kThreads) {
+      for (int c = tid; c < K / 8; c += blockDim.x) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(g) + c);
         float4 a = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
         float4 b = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
@@ -178,14 +181,14 @@ __device__ __forceinline__ void stage_rows(float* xs, float* xsum, int K, int nb
         reinterpret_cast<float4*>(dst)[2 * c + 1] = b;
       }
     } else {
-      for (int c = tid; c < K / 4; c += kThreads)
+      for (int c = tid; c < K / 4; c += blockDim.x)
         reinterpret_cast<float4*>(dst)[c] = __ldcg(reinterpret_cast<const float4*>(g) + c);
     }
   }
   if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) {
     __syncthreads();
     const int nchunk = K / 32;
-    for (int t = tid; t < nb * nchunk; t += kThreads) {
+    for (int t = tid; t < nb * nchunk; t += blockDim.x) {
       const int j = t / nchunk, c = t - j * nchunk;
       const float* s = xs + (size_t)j * K + c * 32;
       float a = 0.f;

@@ -14,27 +14,6 @@
 
 namespace moe {
 
-template <bool XBF16>
-__device__ __forceinline__ float dot_chunk16(uint4 w, uint4 x) {
-  if constexpr (XBF16) {
-    float a = bf16lo(w.x) * bf16lo(x.x);
-    a = fmaf(bf16hi(w.x), bf16hi(x.x), a);
-    a = fmaf(bf16lo(w.y), bf16lo(x.y), a);
-    a = fmaf(bf16hi(w.y), bf16hi(x.y), a);
-    a = fmaf(bf16lo(w.z), bf16lo(x.z), a);
-    a = fmaf(bf16hi(w.z), bf16hi(x.z), a);
-    a = fmaf(bf16lo(w.w), bf16lo(x.w), a);
-    a = fmaf(bf16hi(w.w), bf16hi(x.w), a);
-    return a;
-  } else {
-    float a = __uint_as_float(w.x) * __uint_as_float(x.x);
-    a = fmaf(__uint_as_float(w.y), __uint_as_float(x.y), a);
-    a = fmaf(__uint_as_float(w.z), __uint_as_float(x.z), a);
-    a = fmaf(__uint_as_float(w.w), __uint_as_float(x.w), a);
-    return a;
-  }
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -46,6 +25,37 @@ __device__ __forceinline__ float warp_max(float v) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
+
+// One router dot product by one warp: lane l takes 16-byte chunks l, l+32, ... of the router
+// row, xchunk(c, xv) supplies the chunk's activations as fp32, then a butterfly warp sum. Both
+// launch paths use this, so a logit's bits do not depend on which path (or m) computed it.
+template <bool XBF16, typename XChunk>
+__device__ __forceinline__ float router_dot_warp(const uint8_t* row, int nch, XChunk xchunk) {
+  const int lane = threadIdx.x & 31;
+  float acc = 0.f;
+  for (int c = lane; c < nch; c += 32) {
+    const uint4 w = ldg_stream(row + (size_t)c * 16);
+    float xv[8];
+    xchunk(c, xv);
+    if constexpr (XBF16) {
+      acc = fmaf(bf16lo(w.x), xv[0], acc);
+      acc = fmaf(bf16hi(w.x), xv[1], acc);
+      acc = fmaf(bf16lo(w.y), xv[2], acc);
+      acc = fmaf(bf16hi(w.y), xv[3], acc);
+      acc = fmaf(bf16lo(w.z), xv[4], acc);
+      acc = fmaf(bf16hi(w.z), xv[5], acc);
+      acc = fmaf(bf16lo(w.w), xv[6], acc);
+      acc = fmaf(bf16hi(w.w), xv[7], acc);
+    } else {
+      acc = fmaf(__uint_as_float(w.x), xv[0], acc);
+      acc = fmaf(__uint_as_float(w.y), xv[1], acc);
+      acc = fmaf(__uint_as_float(w.z), xv[2], acc);
+      acc = fmaf(__uint_as_float(w.w), xv[3], acc);
+    }
+  }
+  return warp_sum(acc);
+}
+
 
 // Routing of row r by one warp: selection keys, k rounds of warp arg-max (ties to the lower
 // id), weights. Writes idx / wts (global) and s_idx (shared).
@@ -208,38 +218,25 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_group_kernel(
   const uint8_t* wrow = erow < p.E ? (const uint8_t*)p.router_w + (size_t)erow * row_bytes
                                    : (const uint8_t*)p.shared_gate_w;
   const uint8_t* xb = (const uint8_t*)p.x;
-  __shared__ float s_red[kRouterThreads / 32][8];
   __shared__ int s_last;
   __shared__ int s_idx[MOE_MAX_ROWS * MOE_MAX_TOP_K];
 
-  for (int rb = 0; rb < p.m; rb += 8) {
-    float acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-    for (int c = tid; c < nch; c += kRouterThreads) {
-      const uint4 w = ldg_stream(wrow + (size_t)c * 16);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (rb + j < p.m) {
-          const uint4 xv = __ldg((const uint4*)(xb + (size_t)(rb + j) * row_bytes) + c);
-          acc[j] += dot_chunk16<XBF16>(w, xv);
-        }
+  // one warp per activation row; the router row comes from L2 after the first warp's pass
+  for (int r = warp; r < p.m; r += kRouterThreads / 32) {
+    const uint8_t* xr = xb + (size_t)r * row_bytes;
+    const float acc = router_dot_warp<XBF16>(wrow, nch, [&](int c, float* xv) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr) + c);
+      if constexpr (XBF16) {
+        xv[0] = bf16lo(v.x); xv[1] = bf16hi(v.x); xv[2] = bf16lo(v.y); xv[3] = bf16hi(v.y);
+        xv[4] = bf16lo(v.z); xv[5] = bf16hi(v.z); xv[6] = bf16lo(v.w); xv[7] = bf16hi(v.w);
+      } else {
+        xv[0] = __uint_as_float(v.x); xv[1] = __uint_as_float(v.y);
+        xv[2] = __uint_as_float(v.z); xv[3] = __uint_as_float(v.w);
       }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float v = warp_sum(acc[j]);
-      if (lane == 0) s_red[warp][j] = v;
-    }
-    __syncthreads();
-    if (tid < 8 && rb + tid < p.m) {
-      float v = 0.f;
-#pragma unroll
-      for (int w = 0; w < kRouterThreads / 32; ++w) v += s_red[w][tid];
-      p.logits[(size_t)(rb + tid) * (p.E + 1) + erow] = v;
-    }
-    __syncthreads();
+    });
+    if (lane == 0) p.logits[(size_t)r * (p.E + 1) + erow] = acc;
   }
+  __syncthreads();
 
   if (tid == 0) {
     __threadfence();

@@ -196,3 +196,48 @@ def test_cuda_graph_replay_matches_eager():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(eager, graphed)
+
+
+# ---- the two launch paths: one persistent kernel (m <= 4) and the three-kernel chain --------
+
+class _Path:
+    def __init__(self, name):
+        self.name = name
+
+    def __enter__(self):
+        import os
+        self.old = os.environ.get("MOE_DECODE_PATH")
+        if self.name == "chain":
+            os.environ["MOE_DECODE_PATH"] = "chain"
+        else:
+            os.environ.pop("MOE_DECODE_PATH", None)
+
+    def __exit__(self, *a):
+        import os
+        if self.old is None:
+            os.environ.pop("MOE_DECODE_PATH", None)
+        else:
+            os.environ["MOE_DECODE_PATH"] = self.old
+
+
+PATH_CASES = [(n, m) for n in ("qwen3_30b_a3b", "lfm2_8b_a1b", "qwen3_6_35b_a3b", "llama4_scout")
+              for m in (1, 2, 3, 4)] + [(n, m) for n in SMALL for m in (1, 4)]
+
+
+@pytest.mark.parametrize("name,m", PATH_CASES)
+def test_persistent_kernel_and_chain_agree_bitwise(name, m):
+    cfg = SMALL.get(name) or CONFIGS[name]
+    lay, dev, olay = layer_for(cfg)
+    x = lay.x(m, offset=5)
+    with _Path("chain"):
+        chain, rt_c, st_c = run(dev, x)
+    with _Path("auto"):
+        auto, rt_a, st_a = run(dev, x)
+    assert st_c == B.MOE_OK and st_a == B.MOE_OK
+    for key in ("idx", "sorted_pairs", "expert_offsets", "token_to_perm", "active"):
+        np.testing.assert_array_equal(rt_a[key], rt_c[key], err_msg=key)
+    np.testing.assert_array_equal(rt_a["w"], rt_c["w"])
+    np.testing.assert_array_equal(auto, chain)
+    rows = SAMPLE_ROWS.get((name, m))
+    want, _ = ref.moe_forward(olay, x, rows=rows)
+    check_out(auto if rows is None else auto[rows], want)
