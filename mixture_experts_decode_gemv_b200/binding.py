@@ -14,7 +14,8 @@ from typing import Optional
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmoedecode.so")
+# MOE_DECODE_LIBRARY may name another build of the same library (e.g. an instrumented one).
+LIB_PATH = os.environ.get("MOE_DECODE_LIBRARY") or os.path.join(_PKG, "libmoedecode.so")
 
 MOE_OK = 0
 MOE_ERR_NULL_POINTER = -1

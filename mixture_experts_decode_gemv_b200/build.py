@@ -42,12 +42,17 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = False,
+          defines=(), out: str = None) -> str:
+    """Compile the library; ``defines`` (e.g. ``("MOE_PHASE_TIMERS",)``) and ``out`` give a
+    separately named variant build."""
+    target = out or LIB
+    if not force and not defines and out is None and up_to_date():
         return LIB
     cmd = [_nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
            "-cudart", "static", "--expt-relaxed-constexpr", "-I", INCLUDE,
-           "-o", LIB + ".tmp", *[os.path.join(CSRC, s) for s in SOURCES]]
+           *[f"-D{d}" for d in defines],
+           "-o", target + ".tmp", *[os.path.join(CSRC, s) for s in SOURCES]]
     if ptxas_verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     if not quiet:
@@ -57,13 +62,15 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = False)
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if ptxas_verbose or (res.stderr.strip() and not quiet):
         print(res.stderr, file=sys.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(target + ".tmp", target)
+    return target
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--define", action="append", default=[])
+    ap.add_argument("--out", default=None)
     a = ap.parse_args()
-    print(build(force=a.force, ptxas_verbose=a.ptxas_verbose))
+    print(build(force=a.force, ptxas_verbose=a.ptxas_verbose, defines=a.define, out=a.out))

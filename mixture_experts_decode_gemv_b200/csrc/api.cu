@@ -238,16 +238,17 @@ constexpr size_t kFusedSmemBudget = 220 * 1024;
 // Shared-memory plan of the persistent kernel; false when the layer does not fit it.
 bool plan_fused(const moe_cfg& c, int m, bool has_shared, int fmt, int sms, FusedPlan* fp) {
   if (m > kFusedMaxRows || sms <= 0) return false;
+  const int h = c.hidden, I = c.moe_inter, S = has_shared ? c.shared_inter : 0;
   const int te = m * c.top_k, n_rows = te + (has_shared ? m : 0);
-  const int kmax = (has_shared && c.shared_inter > c.moe_inter) ? c.shared_inter : c.moe_inter;
+  const int kmax = S > I ? S : I;
   const int ld = (kmax + 31) / 32 * 32;
-  const int cols = (c.hidden + sms - 1) / sms;
+  const int cols = (h + sms - 1) / sms;
   const bool q4 = fmt == MOE_FMT_Q4_AFFINE_G64;
   size_t off = 0;
   fp->xs_off = (int)off;
-  off += align16((size_t)m * c.hidden * 4);
+  off += align16((size_t)m * h * 4);
   fp->xsum_off = (int)off;
-  off += q4 ? align16((size_t)m * (c.hidden / 32) * 4) : 0;
+  off += q4 ? align16((size_t)m * (h / 32) * 4) : 0;
   fp->act_off = (int)off;
   off += align16((size_t)n_rows * ld * 4);
   fp->actsum_off = (int)off;
@@ -260,12 +261,13 @@ bool plan_fused(const moe_cfg& c, int m, bool has_shared, int fmt, int sms, Fuse
   fp->act_ld = ld;
   fp->smem_bytes = (int)off;
   fp->spin_limit = 2000000000LL;  // about a second of clock cycles
+  fp->l2_prefetch_cap = 48LL << 20;
   return true;
 }
 
 template <int FMT, bool XBF16, int RB>
 cudaError_t launch_fused_t(const Params& p, const FusedPlan& fp, cudaStream_t st) {
-  auto kernel = moe_fused_kernel<FMT, FMT, XBF16, RB>;
+  auto kernel = moe_fused_kernel<FMT, XBF16, RB>;
   static bool attr_done = false;
   {
     static std::mutex mu;

@@ -1,19 +1,19 @@
 // Dequant-fused expert kernels of the decode MoE layer (CUDA-core GEMV-style tiles).
 //
-// gate_up_swiglu_kernel: one CTA = 32 rows i of one expert's gate and up matrices for every pair
-//   routed to that expert (or every row, for the shared expert). 8 lanes share one (gate_i, up_i)
-//   row pair, each lane streaming 16-byte chunks with non-allocating 128-bit loads and decoding
-//   them in registers; the expert's activation rows are staged once in shared memory as fp32 and
-//   read by all 32 row pairs (the 4 row pairs of a warp read the same addresses, a broadcast).
-//   act[pos, i] = silu(g) * u is written per sorted pair position.
+// Every weight row is reduced by one whole warp: lane l takes the row's 16-byte chunks l, l+32,
+// l+64, ... in order, decodes each in registers and accumulates in fp32, then a butterfly warp
+// sum finishes the row. The same arithmetic runs whether the chunks are streamed from global
+// memory (non-allocating 128-bit loads) or from a shared-memory ring, so both launch paths give
+// identical bits. Activation rows are staged once in shared memory as fp32.
+//
+// gate_up_swiglu_kernel: one CTA = 32 (gate_i, up_i) row pairs of one active expert (or of the
+//   shared expert), 4 per warp, for every pair routed to that expert; act[pos, i] = silu(g) * u
+//   per sorted pair position.
 // down_blend_kernel: one CTA = 64 output columns of one active expert's down matrix (or the
-//   shared expert's) for every row that uses it, into per-pair partials; the CTA that completes a
-//   column tile last (atomic ticket, no spinning) blends the tile for every row: the routed slots
-//   in slot order, each times its weight, then gamma times the shared expert.
-// Accumulation is fp32 throughout; activations stay fp32 between the two kernels.
-// The 8-lane reductions are full-warp shuffles, so every guard around them must be uniform
-// across a warp: rows come 4 per warp and I, S (multiples of 4) and h (multiple of 8) keep the
-// `i < N` / `col0 < h` guards warp-uniform (the host refuses other shapes).
+//   shared expert's), 8 per warp taken two at a time, for every row that uses it, into per-pair
+//   partials; the CTA that completes a column tile last (atomic ticket, no spinning) blends the
+//   tile for every row: routed slots in slot order, each times its weight, then gamma times the
+//   shared expert.
 #pragma once
 
 #include <cuda_fp4.h>
@@ -67,9 +67,48 @@ __device__ __forceinline__ RowRef row_ref(const MatDev& M, int e, int row) {
   return r;
 }
 
+// One 16-byte chunk of a weight row plus the scale fields it needs, loaded together so a chunk
+// costs one memory round trip. aux: Q4 -> fp16 scale (low half) and fp16 bias (high half) of the
+// chunk's 64-element group; NVFP4 -> the two E4M3 block scales of its 32 elements.
+struct Chunk {
+  uint4 w;
+  uint32_t aux;
+};
+
+__device__ __forceinline__ uint32_t ldg_u16(const void* p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+// SMEM: the row lives in shared memory (a ring stage); else in global memory.
+template <int FMT, bool SMEM>
+__device__ __forceinline__ Chunk load_chunk(const RowRef& rr, int c) {
+  Chunk k;
+  k.aux = 0;
+  if constexpr (SMEM) {
+    k.w = *reinterpret_cast<const uint4*>(rr.w + (size_t)c * 16);
+    if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) {
+      k.aux = (uint32_t)(*reinterpret_cast<const unsigned short*>(rr.sc + (size_t)(c >> 1) * 2)) |
+              ((uint32_t)(*reinterpret_cast<const unsigned short*>(rr.bi + (size_t)(c >> 1) * 2))
+               << 16);
+    } else if constexpr (FMT == MOE_FMT_NVFP4) {
+      k.aux = *reinterpret_cast<const unsigned short*>(rr.sc + (size_t)c * 2);
+    }
+  } else {
+    k.w = ldg_stream(rr.w + (size_t)c * 16);
+    if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) {
+      k.aux = ldg_u16(rr.sc + (size_t)(c >> 1) * 2) | (ldg_u16(rr.bi + (size_t)(c >> 1) * 2) << 16);
+    } else if constexpr (FMT == MOE_FMT_NVFP4) {
+      k.aux = ldg_u16(rr.sc + (size_t)c * 2);
+    }
+  }
+  return k;
+}
+
 template <int FMT>
-__device__ __forceinline__ void decode(uint4 raw, const RowRef& rr, int c, Dec<FMT>& d) {
-  const uint32_t q[4] = {raw.x, raw.y, raw.z, raw.w};
+__device__ __forceinline__ void decode(const Chunk& ch, Dec<FMT>& d) {
+  const uint32_t q[4] = {ch.w.x, ch.w.y, ch.w.z, ch.w.w};
   if constexpr (FMT == MOE_FMT_F32) {
 #pragma unroll
     for (int t = 0; t < 4; ++t) d.w[t] = __uint_as_float(q[t]);
@@ -85,8 +124,8 @@ __device__ __forceinline__ void decode(uint4 raw, const RowRef& rr, int c, Dec<F
 #pragma unroll
       for (int n = 0; n < 8; ++n)
         d.f[8 * t + n] = __uint_as_float(0x3F800000u | (((q[t] >> (4 * n)) & 0xFu) << 19));
-    const float s = __half2float(__ldg((const __half*)rr.sc + (c >> 1)));
-    const float b = __half2float(__ldg((const __half*)rr.bi + (c >> 1)));
+    const float s = __half2float(__ushort_as_half((unsigned short)(ch.aux & 0xFFFFu)));
+    const float b = __half2float(__ushort_as_half((unsigned short)(ch.aux >> 16)));
     d.s16 = 16.f * s;
     d.bm = b - 16.f * s;
   } else {  // NVFP4: byte j holds elements 2j (low nibble) and 2j+1 (high nibble)
@@ -100,146 +139,242 @@ __device__ __forceinline__ void decode(uint4 raw, const RowRef& rr, int c, Dec<F
         d.v[8 * t + 2 * b] = f.x;
         d.v[8 * t + 2 * b + 1] = f.y;
       }
-    const unsigned short s2 = __ldg((const unsigned short*)(rr.sc) + c);
-    const __half2_raw hs = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)s2, __NV_E4M3);
+    const __half2_raw hs =
+        __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(ch.aux & 0xFFFFu), __NV_E4M3);
     const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&hs));
     d.s0 = sf.x;
     d.s1 = sf.y;
   }
 }
 
-// Dot product of a decoded chunk with the fp32 activations xs[0..kElems) (16-byte aligned).
+// Shared-memory layout of staged activation rows. The lanes of a quarter-warp read the
+// activations of 8 consecutive weight chunks at once; stored plainly, those reads sit a whole
+// chunk apart and pile onto the same banks (8-way for 4-bit chunks of 32 elements). Each row is
+// therefore stored as 4-float quads with the quad index XOR-swizzled per chunk, so a
+// quarter-warp's reads hit 8 different bank groups. The arithmetic order is unchanged.
+template <int FMT>
+__device__ __forceinline__ int x_quad(int q) {  // logical quad -> stored quad
+  if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64 || FMT == MOE_FMT_NVFP4) {
+    return (q & ~7) | ((q ^ (q >> 3)) & 7);                // 8 quads per chunk
+  } else if constexpr (FMT == MOE_FMT_BF16) {
+    return (q & ~1) | ((q ^ (q >> 3)) & 1);                // 2 quads per chunk
+  } else {
+    return q;                                              // 1 quad per chunk
+  }
+}
+
+template <int FMT>
+__device__ __forceinline__ float4 x_load(const float* row, int q) {
+  return *reinterpret_cast<const float4*>(row + 4 * x_quad<FMT>(q));
+}
+
+// Dot product of decoded chunk c with the staged fp32 activation row `row` (swizzled layout).
 // xsum: for Q4, the sum of the chunk's 32 activations.
 template <int FMT>
-__device__ __forceinline__ float dot(const Dec<FMT>& d, const float* xs, float xsum) {
+__device__ __forceinline__ float dot(const Dec<FMT>& d, const float* row, int c, float xsum) {
+  constexpr int kQ = Fmt<FMT>::kElems / 4;  // quads per chunk
   if constexpr (FMT == MOE_FMT_F32 || FMT == MOE_FMT_BF16) {
-    constexpr int N = Fmt<FMT>::kElems;
     float a = 0.f;
 #pragma unroll
-    for (int t = 0; t < N; t += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(xs + t);
-      a = fmaf(d.w[t], x.x, a);
-      a = fmaf(d.w[t + 1], x.y, a);
-      a = fmaf(d.w[t + 2], x.z, a);
-      a = fmaf(d.w[t + 3], x.w, a);
+    for (int i = 0; i < kQ; ++i) {
+      const float4 x = x_load<FMT>(row, c * kQ + i);
+      a = fmaf(d.w[4 * i], x.x, a);
+      a = fmaf(d.w[4 * i + 1], x.y, a);
+      a = fmaf(d.w[4 * i + 2], x.z, a);
+      a = fmaf(d.w[4 * i + 3], x.w, a);
     }
     return a;
   } else if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) {
     float a = 0.f;
 #pragma unroll
-    for (int t = 0; t < 32; t += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(xs + t);
-      a = fmaf(d.f[t], x.x, a);
-      a = fmaf(d.f[t + 1], x.y, a);
-      a = fmaf(d.f[t + 2], x.z, a);
-      a = fmaf(d.f[t + 3], x.w, a);
+    for (int i = 0; i < 8; ++i) {
+      const float4 x = x_load<FMT>(row, c * 8 + i);
+      a = fmaf(d.f[4 * i], x.x, a);
+      a = fmaf(d.f[4 * i + 1], x.y, a);
+      a = fmaf(d.f[4 * i + 2], x.z, a);
+      a = fmaf(d.f[4 * i + 3], x.w, a);
     }
     return fmaf(d.s16, a, d.bm * xsum);
   } else {
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-    for (int t = 0; t < 16; t += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(xs + t);
-      a0 = fmaf(d.v[t], x.x, a0);
-      a0 = fmaf(d.v[t + 1], x.y, a0);
-      a0 = fmaf(d.v[t + 2], x.z, a0);
-      a0 = fmaf(d.v[t + 3], x.w, a0);
+    for (int i = 0; i < 4; ++i) {
+      const float4 x = x_load<FMT>(row, c * 8 + i);
+      a0 = fmaf(d.v[4 * i], x.x, a0);
+      a0 = fmaf(d.v[4 * i + 1], x.y, a0);
+      a0 = fmaf(d.v[4 * i + 2], x.z, a0);
+      a0 = fmaf(d.v[4 * i + 3], x.w, a0);
     }
 #pragma unroll
-    for (int t = 16; t < 32; t += 4) {
-      const float4 x = *reinterpret_cast<const float4*>(xs + t);
-      a1 = fmaf(d.v[t], x.x, a1);
-      a1 = fmaf(d.v[t + 1], x.y, a1);
-      a1 = fmaf(d.v[t + 2], x.z, a1);
-      a1 = fmaf(d.v[t + 3], x.w, a1);
+    for (int i = 4; i < 8; ++i) {
+      const float4 x = x_load<FMT>(row, c * 8 + i);
+      a1 = fmaf(d.v[4 * i], x.x, a1);
+      a1 = fmaf(d.v[4 * i + 1], x.y, a1);
+      a1 = fmaf(d.v[4 * i + 2], x.z, a1);
+      a1 = fmaf(d.v[4 * i + 3], x.w, a1);
     }
     return fmaf(d.s0, a0, d.s1 * a1);
   }
 }
 
-__device__ __forceinline__ float sum8lanes(float v) {
-  v += __shfl_xor_sync(0xffffffffu, v, 1);
-  v += __shfl_xor_sync(0xffffffffu, v, 2);
-  v += __shfl_xor_sync(0xffffffffu, v, 4);
+__device__ __forceinline__ float warp_allsum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-// Shared-memory staging of up to RB activation rows of length K as fp32, plus (Q4) the sum of
-// every 32-element chunk. src(j) gives the global row pointer of staged row j.
-template <int FMT, bool SRC_BF16, int RB, typename SrcFn>
-__device__ __forceinline__ void stage_rows(float* xs, float* xsum, int K, int nb, SrcFn src) {
-  const int tid = threadIdx.x;
-  for (int j = 0; j < nb; ++j) {
-    const uint8_t* g = src(j);
-    float* dst = xs + (size_t)j * K;
-    if constexpr (SRC_BF16) {
-      for (int c = tid; c < K / 8; c += blockDim.x) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(g) + c);
-        float4 a = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
-        float4 b = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
-        reinterpret_cast<float4*>(dst)[2 * c] = a;
-        reinterpret_cast<float4*>(dst)[2 * c + 1] = b;
-      }
-    } else {
-      for (int c = tid; c < K / 4; c += blockDim.x)
-        reinterpret_cast<float4*>(dst)[c] = __ldcg(reinterpret_cast<const float4*>(g) + c);
-    }
-  }
-  if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) {
-    __syncthreads();
-    const int nchunk = K / 32;
-    for (int t = tid; t < nb * nchunk; t += blockDim.x) {
-      const int j = t / nchunk, c = t - j * nchunk;
-      const float* s = xs + (size_t)j * K + c * 32;
-      float a = 0.f;
+// Staging of nb activation rows of length K as fp32 into shared memory (destination pitch
+// `pitch` floats, swizzled for weight format FMT) and, for Q4 weights, the sum of every
+// 32-element chunk (pitch / 32 per row). src(j) is the global address of row j (bf16 or fp32).
+// Threads t0 .. t0 + nt - 1 take part (nt a multiple of 32). Each thread issues up to four
+// 16-byte loads before storing; a chunk's pieces sit in consecutive lanes, so its sum is a fixed
+// shuffle tree over per-piece sequential sums (same bits whichever path or thread count stages).
+template <int FMT, bool SRC_BF16, typename SrcFn>
+__device__ __forceinline__ void stage_rows(float* xs, float* xsum, int K, int pitch, int nb,
+                                           SrcFn src, int t0, int nt) {
+  constexpr int kPer = SRC_BF16 ? 8 : 4;  // elements per 16-byte piece
+  constexpr int kPieces32 = 32 / kPer;    // pieces per 32-element chunk
+  const int npieces = K / kPer;
+  const int total = nb * npieces;
+  const int me = (int)threadIdx.x - t0;
+  for (int base = 0; base < total; base += 4 * nt) {
+    uint4 v[4];
 #pragma unroll
-      for (int u = 0; u < 32; ++u) a += s[u];
-      xsum[j * nchunk + c] = a;
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * nt + me;
+      if (idx < total) {
+        const int j = idx / npieces, c = idx - j * npieces;
+        const uint4* g = reinterpret_cast<const uint4*>(src(j)) + c;
+        v[u] = SRC_BF16 ? __ldg(g) : __ldcg(g);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * nt + me;
+      const bool live = idx < total;
+      const int j = live ? idx / npieces : 0, c = live ? idx - j * npieces : 0;
+      float f[kPer];
+      if (live) {
+        if constexpr (SRC_BF16) {
+          f[0] = bf16lo(v[u].x); f[1] = bf16hi(v[u].x); f[2] = bf16lo(v[u].y);
+          f[3] = bf16hi(v[u].y); f[4] = bf16lo(v[u].z); f[5] = bf16hi(v[u].z);
+          f[6] = bf16lo(v[u].w); f[7] = bf16hi(v[u].w);
+        } else {
+          f[0] = __uint_as_float(v[u].x); f[1] = __uint_as_float(v[u].y);
+          f[2] = __uint_as_float(v[u].z); f[3] = __uint_as_float(v[u].w);
+        }
+        float* dst = xs + (size_t)j * pitch;
+#pragma unroll
+        for (int t = 0; t < kPer; t += 4)
+          *reinterpret_cast<float4*>(dst + 4 * x_quad<FMT>((c * kPer + t) / 4)) =
+              make_float4(f[t], f[t + 1], f[t + 2], f[t + 3]);
+      }
+      if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) {
+        // the loop bounds are uniform over the participating threads: all lanes shuffle
+        float ps = 0.f;
+        if (live) {
+#pragma unroll
+          for (int t = 0; t < kPer; ++t) ps += f[t];
+        }
+#pragma unroll
+        for (int o = 1; o < kPieces32; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        if (live && (c % kPieces32) == 0) xsum[(size_t)j * (pitch / 32) + c / kPieces32] = ps;
+      }
     }
   }
 }
 
-template <int FMT>
-constexpr int unroll_of() { return (FMT == MOE_FMT_F32) ? 4 : 4; }
+// Chunks per lane in flight: deep for global memory (latency), shallow for shared memory and
+// when several activation rows make each chunk's arithmetic longer.
+template <int FMT, bool SMEM, int RB>
+constexpr int row_unroll() {
+  return SMEM ? 2 : (FMT == MOE_FMT_BF16 || FMT == MOE_FMT_F32 ? (RB > 1 ? 4 : 8) : (RB > 1 ? 2 : 4));
+}
 
-// Accumulate two weight rows (A, B) against nb staged rows: acc_a[j], acc_b[j].
-template <int FMT, int RB>
-__device__ __forceinline__ void two_row_dots(const RowRef& A, const RowRef& B, int nch, int lg,
-                                             const float* xs, const float* xsum, int K, int nb,
-                                             float (&acc_a)[RB], float (&acc_b)[RB]) {
-  constexpr int kE = Fmt<FMT>::kElems;
-  constexpr int U = unroll_of<FMT>();
-  const int nchunk32 = K / 32;
-  for (int c0 = lg; c0 < nch; c0 += kLanesPerRow * U) {
-    uint4 ra[U], rb[U];
+// Two weight rows A and B (same length, nch chunks) against nb <= RB activation rows, by one
+// warp: per-lane partial sums in chunk order, then a butterfly sum. xr[j] / xsr[j]: staged row j
+// and (Q4) its chunk sums. acc_a / acc_b receive the full dot products (every lane).
+template <int FMT, int RB, bool SMEM>
+__device__ __forceinline__ void rows2_dot(const RowRef& A, const RowRef& B, int nch,
+                                          const float* const (&xr)[RB],
+                                          const float* const (&xsr)[RB], int nb,
+                                          float (&acc_a)[RB], float (&acc_b)[RB]) {
+  constexpr int U = row_unroll<FMT, SMEM, RB>();
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < RB; ++j) acc_a[j] = acc_b[j] = 0.f;
+  for (int c0 = lane; c0 < nch; c0 += 32 * U) {
+    Chunk ra[U], rb[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int c = c0 + u * kLanesPerRow;
+      const int c = c0 + 32 * u;
       if (c < nch) {
-        ra[u] = ldg_stream(A.w + (size_t)c * 16);
-        rb[u] = ldg_stream(B.w + (size_t)c * 16);
+        ra[u] = load_chunk<FMT, SMEM>(A, c);
+        rb[u] = load_chunk<FMT, SMEM>(B, c);
       }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int c = c0 + u * kLanesPerRow;
+      const int c = c0 + 32 * u;
       if (c < nch) {
         Dec<FMT> da, db;
-        decode<FMT>(ra[u], A, c, da);
-        decode<FMT>(rb[u], B, c, db);
+        decode<FMT>(ra[u], da);
+        decode<FMT>(rb[u], db);
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
           if (j < nb) {
-            const float* x = xs + (size_t)j * K + c * kE;
             float s = 0.f;
-            if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) s = xsum[j * nchunk32 + c];
-            acc_a[j] += dot<FMT>(da, x, s);
-            acc_b[j] += dot<FMT>(db, x, s);
+            if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) s = xsr[j][c];
+            acc_a[j] += dot<FMT>(da, xr[j], c, s);
+            acc_b[j] += dot<FMT>(db, xr[j], c, s);
           }
         }
       }
     }
   }
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    acc_a[j] = warp_allsum(acc_a[j]);
+    acc_b[j] = warp_allsum(acc_b[j]);
+  }
+}
+
+// One weight row (same arithmetic per row as rows2_dot).
+template <int FMT, int RB, bool SMEM>
+__device__ __forceinline__ void rows1_dot(const RowRef& A, int nch,
+                                          const float* const (&xr)[RB],
+                                          const float* const (&xsr)[RB], int nb,
+                                          float (&acc)[RB]) {
+  constexpr int U = row_unroll<FMT, SMEM, RB>();
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < RB; ++j) acc[j] = 0.f;
+  for (int c0 = lane; c0 < nch; c0 += 32 * U) {
+    Chunk ra[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nch) ra[u] = load_chunk<FMT, SMEM>(A, c);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nch) {
+        Dec<FMT> da;
+        decode<FMT>(ra[u], da);
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+          if (j < nb) {
+            float s = 0.f;
+            if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) s = xsr[j][c];
+            acc[j] += dot<FMT>(da, xr[j], c, s);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < RB; ++j) acc[j] = warp_allsum(acc[j]);
 }
 
 template <int FMT, bool XBF16, int RB>
@@ -276,51 +411,51 @@ __global__ void __launch_bounds__(kThreads) gate_up_swiglu_kernel(const __grid_c
     dst = p.act;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int lg = lane & (kLanesPerRow - 1);
-  const int i = tile * kRowsPerCta + warp * kRowsPerWarp + (lane >> 3);
   const int nch = (int)(packed_row_bytes(FMT, K) / 16);
   const size_t xrow_bytes = (size_t)K * (XBF16 ? 2 : 4);
-  RowRef A{}, B{};
-  if (i < N) {
-    A = row_ref<FMT>(*G, e, i);
-    B = row_ref<FMT>(*U, e, i);
+  const float* xr[RB];
+  const float* xsr[RB];
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    xr[j] = xs + (size_t)j * K;
+    xsr[j] = xsum + (size_t)j * (K / 32);
   }
   for (int rb = 0; rb < nrows; rb += RB) {
     const int nb = min(RB, nrows - rb);
-    stage_rows<FMT, XBF16, RB>(xs, xsum, K, nb, [&](int j) {
+    stage_rows<FMT, XBF16>(xs, xsum, K, K, nb, [&](int j) {
       const int r = is_shared ? rb + j : __ldcg(p.sorted_pairs + beg + rb + j) / p.k;
       return (const uint8_t*)p.x + (size_t)r * xrow_bytes;
-    });
+    }, 0, kThreads);
     __syncthreads();
-    if (i < N) {
+    // warp w takes row pairs tile*32 + w*4 + t; the guard is warp-uniform
+    for (int t = 0; t < kRowsPerWarp; ++t) {
+      const int i = tile * kRowsPerCta + warp * kRowsPerWarp + t;
+      if (i >= N) break;
+      const RowRef A = row_ref<FMT>(*G, e, i), B = row_ref<FMT>(*U, e, i);
       float ag[RB], au[RB];
+      rows2_dot<FMT, RB, false>(A, B, nch, xr, xsr, nb, ag, au);
+      if (lane < nb) {
+        float g = 0.f, u = 0.f;
 #pragma unroll
-      for (int j = 0; j < RB; ++j) ag[j] = au[j] = 0.f;
-      two_row_dots<FMT, RB>(A, B, nch, lg, xs, xsum, K, nb, ag, au);
-#pragma unroll
-      for (int j = 0; j < RB; ++j) {
-        ag[j] = sum8lanes(ag[j]);
-        au[j] = sum8lanes(au[j]);
-      }
-      if (lg == 0) {
-#pragma unroll
-        for (int j = 0; j < RB; ++j) {
-          if (j < nb) {
-            float g = ag[j] * A.ts, u = au[j] * B.ts;
-            size_t pos;
-            if (is_shared) {
-              pos = rb + j;
-            } else {
-              pos = beg + rb + j;
-              if (p.before_ffn) {
-                const float w = __ldcg(p.wts + __ldcg(p.sorted_pairs + pos));
-                g *= w;
-                u *= w;
-              }
-            }
-            dst[pos * N + i] = silu_mul(g, u);
+        for (int j = 0; j < RB; ++j)
+          if (j == lane) {
+            g = ag[j];
+            u = au[j];
+          }
+        g *= A.ts;
+        u *= B.ts;
+        size_t pos;
+        if (is_shared) {
+          pos = rb + lane;
+        } else {
+          pos = beg + rb + lane;
+          if (p.before_ffn) {
+            const float w = __ldcg(p.wts + __ldcg(p.sorted_pairs + pos));
+            g *= w;
+            u *= w;
           }
         }
+        dst[pos * N + i] = silu_mul(g, u);
       }
     }
     __syncthreads();
@@ -357,39 +492,37 @@ __global__ void __launch_bounds__(kThreads) down_blend_kernel(const __grid_const
     dst = p.ypart + (size_t)beg * p.h;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int lg = lane & (kLanesPerRow - 1);
-  // each 8-lane group owns two output columns of the tile: col0 and col0 + 32
-  const int col0 = tile * kColsPerCta + warp * kRowsPerWarp + (lane >> 3);
-  const int col1 = col0 + kRowsPerCta;
-  const bool ok0 = col0 < p.h, ok1 = col1 < p.h;
   const int nch = (int)(packed_row_bytes(FMT, K) / 16);
-  RowRef A{}, B{};
-  if (ok0) A = row_ref<FMT>(D, e, col0);
-  B = ok1 ? row_ref<FMT>(D, e, col1) : A;
+  const float* xr[RB];
+  const float* xsr[RB];
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    xr[j] = xs + (size_t)j * K;
+    xsr[j] = xsum + (size_t)j * (K / 32);
+  }
+  constexpr int kColsPerWarp = kColsPerCta / kWarps;  // 8, taken two at a time
   for (int rb = 0; rb < nrows; rb += RB) {
     const int nb = min(RB, nrows - rb);
-    stage_rows<FMT, false, RB>(xs, xsum, K, nb, [&](int j) {
+    stage_rows<FMT, false>(xs, xsum, K, K, nb, [&](int j) {
       return (const uint8_t*)(src + (size_t)(rb + j) * K);
-    });
+    }, 0, kThreads);
     __syncthreads();
-    if (ok0) {
+    for (int t = 0; t < kColsPerWarp; t += 2) {
+      const int col0 = tile * kColsPerCta + warp * kColsPerWarp + t, col1 = col0 + 1;
+      if (col0 >= p.h) break;  // h is a multiple of 8: col1 < h whenever col0 < h
+      const RowRef A = row_ref<FMT>(D, e, col0), B = row_ref<FMT>(D, e, col1);
       float a0[RB], a1[RB];
+      rows2_dot<FMT, RB, false>(A, B, nch, xr, xsr, nb, a0, a1);
+      if (lane < nb) {
+        float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-      for (int j = 0; j < RB; ++j) a0[j] = a1[j] = 0.f;
-      two_row_dots<FMT, RB>(A, B, nch, lg, xs, xsum, K, nb, a0, a1);
-#pragma unroll
-      for (int j = 0; j < RB; ++j) {
-        a0[j] = sum8lanes(a0[j]);
-        a1[j] = sum8lanes(a1[j]);
-      }
-      if (lg == 0) {
-#pragma unroll
-        for (int j = 0; j < RB; ++j) {
-          if (j < nb) {
-            dst[(size_t)(rb + j) * p.h + col0] = a0[j] * A.ts;
-            if (ok1) dst[(size_t)(rb + j) * p.h + col1] = a1[j] * B.ts;
+        for (int j = 0; j < RB; ++j)
+          if (j == lane) {
+            v0 = a0[j];
+            v1 = a1[j];
           }
-        }
+        dst[(size_t)(rb + lane) * p.h + col0] = v0 * A.ts;
+        dst[(size_t)(rb + lane) * p.h + col1] = v1 * B.ts;
       }
     }
     __syncthreads();

@@ -27,55 +27,78 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // One router dot product by one warp: lane l takes 16-byte chunks l, l+32, ... of the router
-// row, xchunk(c, xv) supplies the chunk's activations as fp32, then a butterfly warp sum. Both
-// launch paths use this, so a logit's bits do not depend on which path (or m) computed it.
+// row, xchunk(c, xv) supplies the chunk's activations as fp32, then a butterfly warp sum. The
+// weight loads of up to 8 chunks are issued before any is used. Both launch paths use this, so a
+// logit's bits do not depend on which path (or m) computed it.
 template <bool XBF16, typename XChunk>
 __device__ __forceinline__ float router_dot_warp(const uint8_t* row, int nch, XChunk xchunk) {
   const int lane = threadIdx.x & 31;
   float acc = 0.f;
-  for (int c = lane; c < nch; c += 32) {
-    const uint4 w = ldg_stream(row + (size_t)c * 16);
-    float xv[8];
-    xchunk(c, xv);
-    if constexpr (XBF16) {
-      acc = fmaf(bf16lo(w.x), xv[0], acc);
-      acc = fmaf(bf16hi(w.x), xv[1], acc);
-      acc = fmaf(bf16lo(w.y), xv[2], acc);
-      acc = fmaf(bf16hi(w.y), xv[3], acc);
-      acc = fmaf(bf16lo(w.z), xv[4], acc);
-      acc = fmaf(bf16hi(w.z), xv[5], acc);
-      acc = fmaf(bf16lo(w.w), xv[6], acc);
-      acc = fmaf(bf16hi(w.w), xv[7], acc);
-    } else {
-      acc = fmaf(__uint_as_float(w.x), xv[0], acc);
-      acc = fmaf(__uint_as_float(w.y), xv[1], acc);
-      acc = fmaf(__uint_as_float(w.z), xv[2], acc);
-      acc = fmaf(__uint_as_float(w.w), xv[3], acc);
+  for (int c0 = lane; c0 < nch; c0 += 32 * 8) {
+    uint4 w[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (c0 + 32 * u < nch) w[u] = ldg_stream(row + (size_t)(c0 + 32 * u) * 16);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nch) {
+        float xv[8];
+        xchunk(c, xv);
+        if constexpr (XBF16) {
+          acc = fmaf(bf16lo(w[u].x), xv[0], acc);
+          acc = fmaf(bf16hi(w[u].x), xv[1], acc);
+          acc = fmaf(bf16lo(w[u].y), xv[2], acc);
+          acc = fmaf(bf16hi(w[u].y), xv[3], acc);
+          acc = fmaf(bf16lo(w[u].z), xv[4], acc);
+          acc = fmaf(bf16hi(w[u].z), xv[5], acc);
+          acc = fmaf(bf16lo(w[u].w), xv[6], acc);
+          acc = fmaf(bf16hi(w[u].w), xv[7], acc);
+        } else {
+          acc = fmaf(__uint_as_float(w[u].x), xv[0], acc);
+          acc = fmaf(__uint_as_float(w[u].y), xv[1], acc);
+          acc = fmaf(__uint_as_float(w[u].z), xv[2], acc);
+          acc = fmaf(__uint_as_float(w[u].w), xv[3], acc);
+        }
+      }
     }
   }
   return warp_sum(acc);
 }
 
+// Order-preserving map of a float key to uint32 (NaN ranks as -infinity).
+__device__ __forceinline__ uint32_t key_bits(float v) {
+  if (v != v) v = -INFINITY;
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 
-// Routing of row r by one warp: selection keys, k rounds of warp arg-max (ties to the lower
-// id), weights. Writes idx / wts (global) and s_idx (shared).
-__device__ void route_row_warp(const Params& p, int r, int* s_idx) {
+// Routing of row r by one warp. Lane s < k ends with the s-th selected expert (descending key,
+// ties to the lower id) and its weight; every lane gets gamma (shared-expert gate, or 1).
+// Each of the k rounds is a lane-local arg-max over the lane's 8 candidates followed by two
+// warp reductions (max key, then min id among lanes holding that key). Returns false when a
+// selected key is not a finite number.
+__device__ __forceinline__ bool route_row(const Params& p, int r, int& my_id, float& my_w,
+                                          float& gamma) {
   const int lane = threadIdx.x & 31;
   const int E = p.E, k = p.k;
   const float* lrow = p.logits + (size_t)r * (E + 1);
-  float lg[8], key[8];
+  float lg[8];
+  uint32_t key[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int e = lane + 32 * j;
-    const bool valid = e < E;
-    const float l = valid ? __ldcg(lrow + e) : -INFINITY;
-    lg[j] = l;
-    float kv = l;
+    lg[j] = e < E ? __ldcg(lrow + e) : -INFINITY;
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane + 32 * j;
+    float kv = lg[j];
     if (p.routing == MOE_ROUTE_SIGMOID && !p.raw) {
-      kv = 1.0f / (1.0f + expf(-l));
-      if (p.has_bias && valid) kv += __ldg(p.expert_bias + e);
+      kv = 1.0f / (1.0f + expf(-lg[j]));
+      if (p.has_bias && e < E) kv += __ldg(p.expert_bias + e);
     }
-    key[j] = valid ? kv : -INFINITY;
+    key[j] = e < E ? key_bits(kv) : 0u;
   }
   float mx = -INFINITY, den = 0.f;
   if (p.routing == MOE_ROUTE_SOFTMAX) {
@@ -87,62 +110,62 @@ __device__ void route_row_warp(const Params& p, int r, int* s_idx) {
     den = warp_sum(den);
   }
   unsigned taken = 0;
-  int my_id = 0;
+  bool ok = true;
+  my_id = 0;
   float my_l = 0.f;
-  bool bad = false;
   for (int s = 0; s < k; ++s) {
-    float bk = -INFINITY;
-    int bid = 0x7fffffff;
-    float bl = 0.f;
+    uint32_t bk = 0;
+    int bj = -1;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E && !((taken >> j) & 1u) && (key[j] > bk || (key[j] == bk && e < bid))) {
+    for (int j = 0; j < 8; ++j) {  // ascending ids within the lane: strict > keeps the lowest
+      if (!((taken >> j) & 1u) && lane + 32 * j < E && (bj < 0 || key[j] > bk)) {
         bk = key[j];
-        bid = e;
-        bl = lg[j];
+        bj = j;
       }
     }
+    const uint32_t best = __reduce_max_sync(0xffffffffu, bj >= 0 ? bk : 0u);
+    const uint32_t cand = (bj >= 0 && bk == best) ? (uint32_t)(lane + 32 * bj) : 0xFFFFFFFFu;
+    const uint32_t id = __reduce_min_sync(0xffffffffu, cand);
+    const int owner = (int)(id & 31u);
+    float l = 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
-      const float ol = __shfl_xor_sync(0xffffffffu, bl, o);
-      if (ok > bk || (ok == bk && oid < bid)) {
-        bk = ok;
-        bid = oid;
-        bl = ol;
-      }
-    }
-    if (bid >= E) {  // only NaN keys left: keep every index in range and flag the row
-      bad = true;
-      bid = s;
-    }
-    if ((bid & 31) == lane) taken |= 1u << (bid >> 5);
+    for (int j = 0; j < 8; ++j)
+      if (lane == owner && (int)(id >> 5) == j) l = lg[j];
+    l = __shfl_sync(0xffffffffu, l, owner);
+    if (lane == owner) taken |= 1u << (id >> 5);
+    if (best <= key_bits(-INFINITY)) ok = false;  // -inf or NaN won a slot
     if (lane == s) {
-      my_id = bid;
-      my_l = bl;
+      my_id = (int)id;
+      my_l = l;
     }
   }
   float wv = 0.f;
-  if (lane < k) {
+  if (lane < k)
     wv = (p.routing == MOE_ROUTE_SOFTMAX) ? expf(my_l - mx) / den : 1.0f / (1.0f + expf(-my_l));
-  }
   if (p.norm) {
     const float tot = warp_sum(lane < k ? wv : 0.f);
     wv = wv / tot;
   }
-  wv *= p.rsf;
-  if (lane < k) {
-    p.idx[r * k + lane] = my_id;
-    p.wts[r * k + lane] = wv;
-    s_idx[r * k + lane] = my_id;
+  my_w = wv * p.rsf;
+  gamma = 1.f;
+  if (p.shared_kind == MOE_SHARED_SIGMOID_GATE) gamma = 1.0f / (1.0f + expf(-__ldcg(lrow + E)));
+  return ok;
+}
+
+// Routing of row r for the multi-kernel path: route_row, then the global and shared writes.
+__device__ void route_row_warp(const Params& p, int r, int* s_idx) {
+  const int lane = threadIdx.x & 31;
+  int id;
+  float w, g;
+  const bool ok = route_row(p, r, id, w, g);
+  if (lane < p.k) {
+    p.idx[r * p.k + lane] = id;
+    p.wts[r * p.k + lane] = w;
+    s_idx[r * p.k + lane] = id;
   }
   if (lane == 0) {
-    if (p.shared_kind == MOE_SHARED_SIGMOID_GATE) {
-      p.gamma[r] = 1.0f / (1.0f + expf(-__ldcg(lrow + E)));
-    }
-    if (bad) atomicExch(p.ctrl + kStatus, (unsigned)MOE_ERR_DEVICE_CHECK);
+    if (p.shared_kind == MOE_SHARED_SIGMOID_GATE) p.gamma[r] = g;
+    if (!ok) atomicExch(p.ctrl + kStatus, (unsigned)MOE_ERR_DEVICE_CHECK);
   }
 }
 
