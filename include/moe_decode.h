@@ -154,6 +154,15 @@ int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, const void* rou
                        const moe_expert_table* shared, const void* shared_gate_w, void* out,
                        void* workspace, size_t workspace_bytes, void* stream);
 
+/* Number of kernel launches moe_decode_forward makes for this cfg, m and weight tables on the
+ * current device, into *launches: 1 when the whole call runs as one persistent kernel (m <= 4,
+ * one weight format for every projection, activations within the kernel's shared memory), else
+ * 3 to 5 (router, gate/up and down, the last two split when the shared expert has its own
+ * format). The tables are validated as in moe_decode_forward; nothing is launched. For callers
+ * that budget graph nodes or count launches; the decode pages have no counterpart. */
+int moe_decode_launches(const moe_cfg* cfg, int m, const moe_expert_table* routed,
+                        const moe_expert_table* shared, int* launches);
+
 /* Copy the routing and grouping of the last forward call that used `workspace` to host arrays
  * (synchronises `stream`). Any output pointer may be NULL to skip it. Sizes: idx, weights,
  * sorted_pairs, token_to_perm: m*top_k; expert_offsets: num_experts+1; active: min(m*top_k, E);

@@ -48,7 +48,7 @@ EXPORTS = (
     "moe_workspace_bytes", "moe_workspace_init", "moe_decode_forward", "moe_decode_read_routing",
     "moe_get_device_status", "moe_packed_bytes", "moe_pack_bf16", "moe_quantize_q4_affine",
     "moe_quantize_nvfp4", "moe_dequantize", "moe_status_string", "moe_last_cuda_error",
-    "moe_version", "moe_decode_forward_no_alloc",
+    "moe_version", "moe_decode_forward_no_alloc", "moe_decode_launches",
 )
 
 MOE_NO_ALLOC_SCRATCH_BYTES = 16 << 20
@@ -110,6 +110,8 @@ def _load() -> ctypes.CDLL:
         "moe_dequantize": [i32, vp, vp, vp, vp, i32, i32, vp],
         "moe_decode_forward_no_alloc": [P(moe_cfg), i32, vp, vp, vp, P(moe_expert_table),
                                         P(moe_expert_table), vp, vp, vp],
+        "moe_decode_launches": [P(moe_cfg), i32, P(moe_expert_table), P(moe_expert_table),
+                                P(ctypes.c_int32)],
         "moe_status_string": [i32],
         "moe_last_cuda_error": [],
         "moe_version": [],
@@ -185,6 +187,17 @@ def moe_decode_forward_no_alloc(cfg: moe_cfg, m: int, x, router_w, expert_bias,
         ctypes.byref(shared) if shared is not None else None, _ptr(shared_gate_w), _ptr(out),
         _stream(stream))
     _check(rc, "moe_decode_forward_no_alloc")
+
+
+def moe_decode_launches(cfg: moe_cfg, m: int, routed: moe_expert_table,
+                        shared: Optional[moe_expert_table]) -> int:
+    """Kernel launches one moe_decode_forward call makes on the current device."""
+    n = ctypes.c_int32(0)
+    rc = lib.moe_decode_launches(ctypes.byref(cfg), m, ctypes.byref(routed),
+                                 ctypes.byref(shared) if shared is not None else None,
+                                 ctypes.byref(n))
+    _check(rc, "moe_decode_launches")
+    return int(n.value)
 
 
 def moe_decode_read_routing(cfg: moe_cfg, m: int, workspace, workspace_bytes: int, stream=None):

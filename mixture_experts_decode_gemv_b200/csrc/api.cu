@@ -256,6 +256,23 @@ bool plan_fused(const moe_cfg& c, int m, bool has_shared, int fmt, int sms, Fuse
   fp->y_off = (int)off;
   off += align16((size_t)n_rows * cols * 4);
   if (off > kFusedSmemBudget) return false;
+  // down-row tile: as many phase-E slots (column block of one expert's down rows, with their
+  // scale rows) as the rest of the budget holds, up to every slot a call can have
+  const size_t prb = fmt == MOE_FMT_F32 ? (size_t)kmax * 4
+                     : fmt == MOE_FMT_BF16 ? (size_t)kmax * 2 : (size_t)kmax / 2;
+  const size_t srb = q4 ? (size_t)(kmax / 64) * 2 : fmt == MOE_FMT_NVFP4 ? (size_t)(kmax / 16) : 0;
+  const size_t wblk = align16(cols * prb), sblk = align16(cols * srb);
+  const size_t slot_bytes = wblk + (q4 ? 2 * sblk : sblk);
+  const int max_slots = (c.top_k * m < c.num_experts ? c.top_k * m : c.num_experts) +
+                        (has_shared ? 1 : 0);
+  size_t n_fit = (kFusedSmemBudget - off) / slot_bytes;
+  if (n_fit > (size_t)max_slots) n_fit = (size_t)max_slots;
+  fp->tile_off = (int)off;
+  fp->tile_slots = (int)n_fit;
+  fp->tile_slot_bytes = (int)slot_bytes;
+  fp->tile_sc_off = (int)wblk;
+  fp->tile_bi_off = (int)(wblk + sblk);
+  off += n_fit * slot_bytes;
   fp->grid = sms;
   fp->cols_per_cta = cols;
   fp->act_ld = ld;
@@ -342,6 +359,26 @@ extern "C" int moe_workspace_init(void* workspace, size_t workspace_bytes, void*
   return e == cudaSuccess ? MOE_OK : cuda_fail(e);
 }
 
+// Host dispatch: one persistent kernel for decode-sized calls when every projection shares a
+// format and the call's activations fit in shared memory; the three-kernel chain otherwise.
+bool use_fused(const moe_cfg& c, int m, const moe_expert_table* routed,
+               const moe_expert_table* shared, bool has_shared, FusedPlan* fp) {
+  const int fmt = routed->gate.format;
+  const bool one_fmt = routed->down.format == fmt &&
+                       (!has_shared || (shared->gate.format == fmt && shared->down.format == fmt));
+  return forced_path() != 1 && one_fmt &&
+         fused_formats_ok(fmt, c.x_dtype == MOE_FMT_BF16) &&
+         plan_fused(c, m, has_shared, fmt, sm_count(), fp);
+}
+
+// Launches of the chain: router, gate/up (two when the shared expert has its own format), down
+// (likewise).
+int chain_launches(const moe_expert_table* routed, const moe_expert_table* shared, bool has_shared) {
+  const bool split_gu = has_shared && shared->gate.format != routed->gate.format;
+  const bool split_d = has_shared && shared->down.format != routed->down.format;
+  return 1 + (split_gu ? 2 : 1) + (split_d ? 2 : 1);
+}
+
 extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, const void* router_w,
                                   const float* expert_bias, const moe_expert_table* routed,
                                   const moe_expert_table* shared, const void* shared_gate_w,
@@ -417,17 +454,10 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
   cudaStream_t st = (cudaStream_t)stream;
   const bool xbf16 = c.x_dtype == MOE_FMT_BF16;
 
-  // Host dispatch: one persistent kernel for decode-sized calls when every projection shares a
-  // format and the call's activations fit in shared memory; the three-kernel chain otherwise.
   {
-    const int fmt = routed->gate.format;
-    const bool one_fmt = routed->down.format == fmt &&
-                         (!has_shared || (shared->gate.format == fmt && shared->down.format == fmt));
     FusedPlan fp;
-    const int force = forced_path();
-    if (force != 1 && one_fmt && fused_formats_ok(fmt, xbf16) &&
-        plan_fused(c, m, has_shared, fmt, sm_count(), &fp)) {
-      const cudaError_t e = launch_fused(fmt, xbf16, m, p, fp, st);
+    if (use_fused(c, m, routed, shared, has_shared, &fp)) {
+      const cudaError_t e = launch_fused(routed->gate.format, xbf16, m, p, fp, st);
       return e == cudaSuccess ? MOE_OK : cuda_fail(e);
     }
   }
@@ -480,6 +510,24 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
     e = down(fmt_d, p, p.n_tiles_c * (p.cap + p.has_shared), kmax);
   }
   if (e != cudaSuccess) return cuda_fail(e);
+  return MOE_OK;
+}
+
+extern "C" int moe_decode_launches(const moe_cfg* cfg, int m, const moe_expert_table* routed,
+                                   const moe_expert_table* shared, int* launches) {
+  int rc = check_cfg(cfg, m);
+  if (rc) return rc;
+  if (!launches) return MOE_ERR_NULL_POINTER;
+  const bool has_shared = cfg->shared_kind != MOE_SHARED_NONE;
+  MatDev g, u, d;
+  if ((rc = check_table(routed, cfg->moe_inter, cfg->hidden, cfg->num_experts, &g, &u, &d)))
+    return rc;
+  if (has_shared && (rc = check_table(shared, cfg->shared_inter, cfg->hidden, 1, &g, &u, &d)))
+    return rc;
+  if ((rc = check_device())) return rc;
+  FusedPlan fp;
+  *launches = use_fused(*cfg, m, routed, shared, has_shared, &fp)
+                  ? 1 : chain_launches(routed, shared, has_shared);
   return MOE_OK;
 }
 

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -34,6 +35,23 @@ struct MatDev {
   int fmt;
   int n, k;            // rows and columns of one expert matrix
 };
+
+// Field-wise choice between two matrix descriptors of the kernel parameters. Each field stays a
+// constant-bank read; binding a reference to either descriptor at run time would read the
+// fields through a generic pointer, from memory.
+__device__ __forceinline__ MatDev pick_mat(bool first, const MatDev& a, const MatDev& b) {
+  MatDev r;
+  r.packed = first ? a.packed : b.packed;
+  r.scales = first ? a.scales : b.scales;
+  r.biases = first ? a.biases : b.biases;
+  r.tscale = first ? a.tscale : b.tscale;
+  r.estride = first ? a.estride : b.estride;
+  r.sstride = first ? a.sstride : b.sstride;
+  r.fmt = first ? a.fmt : b.fmt;
+  r.n = first ? a.n : b.n;
+  r.k = first ? a.k : b.k;
+  return r;
+}
 
 // Byte offsets of the workspace regions (all 256-byte aligned).
 struct WsLayout {
@@ -104,11 +122,20 @@ struct Params {
 // ---- PTX helpers -------------------------------------------------------------------------------
 
 // Streaming 16-byte load of weights: read-only path, no L1 allocation.
+// L2 policy for weights that one call reads once: evict them first, so that streaming them does
+// not push out what the next call needs again soon (its code and parameters, the router rows,
+// activations, the routing workspace). No side effects: the compiler may hoist or merge it.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
+               : "l"(p), "l"(l2_evict_first()));
   return r;
 }
 
@@ -125,5 +152,39 @@ __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v &
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + __expf(-z)); }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+// Optional phase timestamps (build with -DMOE_PHASE_TIMERS): thread 0 of every CTA records
+// the SM cycle counter at each phase boundary into the (otherwise unused) down-partials region
+// of the workspace, as uint64 [cta][kPhaseSlots]; slot kPhaseSlots - 1 holds %globaltimer at
+// entry, to line the CTAs up. MOE_STAMP_AFTER(slot, v) reads the counter only once the 32-bit
+// value v has been computed.
+constexpr int kPhaseSlots = 20;
+#ifdef MOE_PHASE_TIMERS
+#define MOE_STAMP_AFTER(slot, v)                                                            \
+  do {                                                                                      \
+    if (threadIdx.x == 0) {                                                                 \
+      unsigned long long t_;                                                                \
+      asm volatile("{ .reg .u32 d_; mov.u32 d_, %1; mov.u64 %0, %%clock64; }"               \
+                   : "=l"(t_) : "r"((unsigned)(v)) : "memory");                              \
+      reinterpret_cast<unsigned long long*>(p.ypart)[blockIdx.x * kPhaseSlots + (slot)] = t_; \
+    }                                                                                       \
+  } while (0)
+#define MOE_STAMP_GLOBAL()                                                                  \
+  do {                                                                                      \
+    if (threadIdx.x == 0) {                                                                 \
+      unsigned long long t_;                                                                \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_)::"memory");                      \
+      reinterpret_cast<unsigned long long*>(p.ypart)[blockIdx.x * kPhaseSlots + kPhaseSlots - 1] = t_; \
+    }                                                                                       \
+  } while (0)
+#else
+#define MOE_STAMP_AFTER(slot, v) \
+  do {                           \
+  } while (0)
+#define MOE_STAMP_GLOBAL() \
+  do {                     \
+  } while (0)
+#endif
+#define MOE_STAMP(slot) MOE_STAMP_AFTER(slot, 0u)
 
 }  // namespace moe

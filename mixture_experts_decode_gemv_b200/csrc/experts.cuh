@@ -77,11 +77,12 @@ struct Chunk {
 
 __device__ __forceinline__ uint32_t ldg_u16(const void* p) {
   unsigned short v;
-  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  asm volatile("ld.global.nc.L2::cache_hint.u16 %0, [%1], %2;" : "=h"(v) : "l"(p), "l"(l2_evict_first()));
   return v;
 }
 
-// SMEM: the row lives in shared memory (a ring stage); else in global memory.
+// SMEM: plain loads (the row may live in shared memory or in L2-resident global memory);
+// else streaming non-allocating global loads.
 template <int FMT, bool SMEM>
 __device__ __forceinline__ Chunk load_chunk(const RowRef& rr, int c) {
   Chunk k;
@@ -284,11 +285,12 @@ __device__ __forceinline__ void stage_rows(float* xs, float* xsum, int K, int pi
   }
 }
 
-// Chunks per lane in flight: deep for global memory (latency), shallow for shared memory and
-// when several activation rows make each chunk's arithmetic longer.
-template <int FMT, bool SMEM, int RB>
+// Chunks per lane in flight: deep for streamed rows (latency; shallower when a chunk holds 32
+// elements or several activation rows make each chunk's arithmetic longer), shallow for plain
+// loads of rows already in shared memory or L2 (short latency, and a smaller loop body).
+template <int FMT, bool PLAIN, int RB>
 constexpr int row_unroll() {
-  return SMEM ? 2 : (FMT == MOE_FMT_BF16 || FMT == MOE_FMT_F32 ? (RB > 1 ? 4 : 8) : (RB > 1 ? 2 : 4));
+  return PLAIN ? 2 : (FMT == MOE_FMT_BF16 || FMT == MOE_FMT_F32 ? (RB > 1 ? 4 : 8) : (RB > 1 ? 2 : 4));
 }
 
 // Two weight rows A and B (same length, nch chunks) against nb <= RB activation rows, by one
@@ -386,13 +388,11 @@ __global__ void __launch_bounds__(kThreads) gate_up_swiglu_kernel(const __grid_c
   float* xsum = smem + (size_t)RB * K;
   const bool is_shared = (int)blockIdx.x < p.n_tiles_s;
   int tile, e = 0, beg = 0, nrows, N;
-  const MatDev* G;
-  const MatDev* U;
+  const MatDev G = pick_mat(is_shared, p.sg, p.rg);
+  const MatDev U = pick_mat(is_shared, p.su, p.ru);
   float* dst;
   if (is_shared) {
     tile = blockIdx.x;
-    G = &p.sg;
-    U = &p.su;
     N = p.S;
     nrows = p.m;
     dst = p.act_sh;
@@ -405,8 +405,6 @@ __global__ void __launch_bounds__(kThreads) gate_up_swiglu_kernel(const __grid_c
     e = __ldcg(p.active + a);
     beg = __ldcg(p.offsets + e);
     nrows = __ldcg(p.offsets + e + 1) - beg;
-    G = &p.rg;
-    U = &p.ru;
     N = p.I;
     dst = p.act;
   }
@@ -431,7 +429,7 @@ __global__ void __launch_bounds__(kThreads) gate_up_swiglu_kernel(const __grid_c
     for (int t = 0; t < kRowsPerWarp; ++t) {
       const int i = tile * kRowsPerCta + warp * kRowsPerWarp + t;
       if (i >= N) break;
-      const RowRef A = row_ref<FMT>(*G, e, i), B = row_ref<FMT>(*U, e, i);
+      const RowRef A = row_ref<FMT>(G, e, i), B = row_ref<FMT>(U, e, i);
       float ag[RB], au[RB];
       rows2_dot<FMT, RB, false>(A, B, nch, xr, xsr, nb, ag, au);
       if (lane < nb) {
@@ -476,7 +474,7 @@ __global__ void __launch_bounds__(kThreads) down_blend_kernel(const __grid_const
   const int K = is_shared ? p.S : p.I;
   float* xs = smem;
   float* xsum = smem + (size_t)RB * K;
-  const MatDev& D = is_shared ? p.sd : p.rd;
+  const MatDev D = pick_mat(is_shared, p.sd, p.rd);
   int e = 0, nrows;
   const float* src;
   float* dst;

@@ -42,6 +42,11 @@ struct FusedPlan {
   int actsum_off;     // Q4 down: per-32 sums of the staged act rows
   int y_off;          // y[(te + m) * cols_per_cta]
   int act_ld;         // row pitch (floats) of the staged act rows
+  int tile_off;       // down-row tile: slot s of phase E at tile_off + s * tile_slot_bytes
+  int tile_slots;     // slots the tile region holds (0: no tile)
+  int tile_slot_bytes;
+  int tile_sc_off;    // within a slot: scales rows, then (Q4) biases rows at 2 * tile_sc_off -
+  int tile_bi_off;    //   packed rows first, each block 16-byte aligned
   int smem_bytes;
   long long spin_limit;       // clock cycles a barrier wait may spin before it gives up
   long long l2_prefetch_cap;  // largest per-call down-projection byte count asked into L2
@@ -70,6 +75,54 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
   unsigned long long v;
   asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
+}
+
+// Shared-memory transaction barrier fed by bulk copies (one phase per launch).
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// Bounded wait for phase `parity` of bar; false when `limit` clock cycles passed first.
+__device__ __forceinline__ bool mbar_wait_bounded(unsigned long long* bar, unsigned parity,
+                                                  long long limit) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > limit) return false;
+  return true;
+}
+// Global -> shared bulk copy (addresses 16-byte aligned, bytes a multiple of 16) completing as
+// transaction bytes on bar; the source lines are marked evict-first in L2 (read once).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes,
+                                         unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
+      "%2, [%3], %4;" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(l2_evict_first())
+      : "memory");
 }
 
 
@@ -114,7 +167,7 @@ struct GridBarrier {
 
 // Routing and grouping kept in shared memory by every CTA.
 struct FusedRoute {
-  int idx[kFusedMaxPairs];
+  alignas(16) int idx[kFusedMaxPairs];
   float w[kFusedMaxPairs];
   float gamma[kFusedMaxRows];
   int sorted[kFusedMaxPairs];     // pair ids by (expert, pair)
@@ -123,47 +176,58 @@ struct FusedRoute {
   int slot_beg[kFusedMaxPairs];   // first position of each active expert in `sorted`
   int slot_n[kFusedMaxPairs];     // its number of pairs
   int n_active;
+  float bias[MOE_MAX_EXPERTS];    // expert biases, staged once per call
+  float ts[kFusedMaxPairs + 1];   // NVFP4 tensor scale of each phase-E slot's down matrix
 };
 
 // Route row r (one warp) into the CTA's shared routing tables (same rule and arithmetic as the
-// multi-kernel path).
-__device__ void fused_route_row(const Params& p, int r, FusedRoute& R) {
+// multi-kernel path). Kept out of line so its per-lane candidate arrays get registers of their
+// own instead of competing with the streaming loops of the kernel around it.
+// With `dry` set it runs the same instructions on any readable rows and stores nothing: an idle
+// warp calls it that way ahead of time, so that the routing code is already in this SM's
+// instruction caches when the real call runs (it runs once per call, after the weights
+// streamed by the previous calls have pushed it out of L2).
+__device__ __noinline__ void fused_route_row(const RouteCfg c, unsigned* status, int r,
+                                             FusedRoute& R, bool dry) {
   const int lane = threadIdx.x & 31;
   int id;
   float w, g;
-  const bool ok = route_row(p, r, id, w, g);
-  if (lane < p.k) {
-    R.idx[r * p.k + lane] = id;
-    R.w[r * p.k + lane] = w;
+  const bool ok = route_row(c, r, R.bias, id, w, g);
+  if (dry) return;
+  if (lane < c.k) {
+    R.idx[r * c.k + lane] = id;
+    R.w[r * c.k + lane] = w;
   }
   if (lane == 0) {
     R.gamma[r] = g;
-    if (!ok) atomicExch(p.ctrl + kStatus, (unsigned)MOE_ERR_DEVICE_CHECK);
+    if (!ok) atomicExch(status, (unsigned)MOE_ERR_DEVICE_CHECK);
   }
 }
 
 // Stable grouping of te <= 32 pairs by expert, by warp 0: pair p (one lane) lands at
 // #(pairs with a smaller expert id) + #(earlier pairs with the same id); the first pair of each
-// expert opens its slot, slots ordered by expert id.
-__device__ void fused_group(const Params& p, FusedRoute& R) {
+// expert opens its slot, slots ordered by expert id. Equal ids come from one match; the counts
+// of smaller ids from every lane reading all te ids (broadcast shared loads).
+__device__ __forceinline__ void fused_group(int te, FusedRoute& R) {
+  constexpr unsigned kFull = 0xffffffffu;
   const int lane = threadIdx.x & 31;
-  const int te = p.m * p.k;
   if (threadIdx.x >= 32) return;
   const bool live = lane < te;
   const int e = live ? R.idx[lane] : 0x7fffffff;
-  int less = 0, eq_before = 0, eq_all = 0;
-  for (int q = 0; q < te; ++q) {
-    const int eq = __shfl_sync(0xffffffffu, e, q);
-    less += eq < e;
-    eq_before += (eq == e) && (q < lane);
-    eq_all += eq == e;
-  }
+  const unsigned same = __match_any_sync(kFull, e);
+  const int eq_before = __popc(same & ((1u << lane) - 1u)), eq_all = __popc(same);
   const bool leader = live && eq_before == 0;
-  const unsigned leaders = __ballot_sync(0xffffffffu, leader);
-  int slot = 0;
-  for (int q = 0; q < te; ++q) {
-    const int eq = __shfl_sync(0xffffffffu, e, q);
-    slot += ((leaders >> q) & 1u) && eq < e;
+  const unsigned leaders = __ballot_sync(kFull, leader);
+  int less = 0, slot = 0;
+  for (int q = 0; q < te; q += 4) {
+    const int4 v = *reinterpret_cast<const int4*>(&R.idx[q]);
+    const int vq[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const bool lt = q + t < te && vq[t] < e;
+      less += lt;
+      slot += lt && ((leaders >> (q + t)) & 1u);
+    }
   }
   if (live) {
     const int pos = less + eq_before;
@@ -179,7 +243,7 @@ __device__ void fused_group(const Params& p, FusedRoute& R) {
 }
 
 // CTA 0 publishes the routing and grouping for read-back (moe_decode_read_routing).
-__device__ void fused_publish(const Params& p, const FusedRoute& R, int nt) {
+__device__ __forceinline__ void fused_publish(const Params& p, const FusedRoute& R, int nt) {
   const int te = p.m * p.k;
   for (int t = threadIdx.x; t < te; t += nt) {
     p.idx[t] = R.idx[t];
@@ -199,24 +263,23 @@ __device__ void fused_publish(const Params& p, const FusedRoute& R, int nt) {
 }
 
 
-// Optional phase timestamps (build with -DMOE_PHASE_TIMERS): thread 0 of every CTA records
-// %globaltimer at each phase boundary into the (otherwise unused) down-partials region of the
-// workspace, as uint64 [cta][kPhaseSlots].
-constexpr int kPhaseSlots = 12;
-#ifdef MOE_PHASE_TIMERS
-#define MOE_STAMP(slot)                                                                     \
-  do {                                                                                      \
-    if (threadIdx.x == 0) {                                                                 \
-      unsigned long long t_;                                                                \
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                \
-      reinterpret_cast<unsigned long long*>(p.ypart)[blockIdx.x * kPhaseSlots + (slot)] = t_; \
-    }                                                                                       \
-  } while (0)
-#else
-#define MOE_STAMP(slot) \
-  do {                  \
-  } while (0)
-#endif
+// Row `lc` (column c0 + lc) of a down matrix held in a shared-memory tile slot.
+template <int FMT>
+__device__ __forceinline__ RowRef tile_row_ref(const MatDev& D, int e, const uint8_t* slot, int K,
+                                               const FusedPlan& fp, int lc) {
+  RowRef r;
+  r.w = slot + (size_t)lc * packed_row_bytes(FMT, K);
+  r.sc = nullptr;
+  r.bi = nullptr;
+  r.ts = 1.f;
+  if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) {
+    r.sc = slot + fp.tile_sc_off + (size_t)lc * (K / 64) * 2;
+    r.bi = slot + fp.tile_bi_off + (size_t)lc * (K / 64) * 2;
+  } else if constexpr (FMT == MOE_FMT_NVFP4) {
+    r.sc = slot + fp.tile_sc_off + (size_t)lc * (K / 16);  // ts: the caller's (staged per slot)
+  }
+  return r;
+}
 
 template <int FMT, bool XBF16, int RB>
 __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
@@ -224,6 +287,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
   extern __shared__ __align__(16) uint8_t fsmem[];
   __shared__ FusedRoute R;
   __shared__ unsigned long long s_base;
+  __shared__ unsigned long long s_tile_bar;   // the down-row tile's bulk copies
+  __shared__ unsigned long long s_tile_mask;  // phase-E slots whose rows sit in the tile
+  __shared__ int s_tile_n;                    // slots offered to the tile
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const int m = p.m, h = p.h, k = p.k, te = m * k;
@@ -243,12 +309,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
   const int ncols = min(h, c0 + fp.cols_per_cta) > c0 ? min(h, c0 + fp.cols_per_cta) - c0 : 0;
   const int nch_h = (int)(packed_row_bytes(FMT, h) / 16);
   MOE_STAMP(0);
+  MOE_STAMP_GLOBAL();
 
   // ---- prologue (may overlap the previous kernel): this CTA's router rows into L2 -----------
   if (tid == 0)
     for (int e = cta; e < e_tot; e += G) prefetch_l2_bulk(router_row(e), xrow_bytes);
   pdl_wait();
   MOE_STAMP(1);
+  if (p.has_bias)
+    for (int e = tid; e < p.E; e += kFusedThreads) R.bias[e] = __ldg(p.expert_bias + e);
   unsigned long long* bar_ctr = reinterpret_cast<unsigned long long*>(p.ctrl + kBarCounter);
   if (tid == 0) s_base = ld_acquire_u64(bar_ctr) / (unsigned long long)G * (unsigned long long)G;
   stage_rows<FMT, XBF16>(xs, xsum, h, h, m, [&](int j) {
@@ -279,6 +348,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
   }
   MOE_STAMP(3);
   bar.arrive();
+  if (warp == kFusedWarps - 4) {  // same scheduler partition as warp 0, which routes row 0
+    RouteCfg dc = route_cfg(p);
+    dc.logits = reinterpret_cast<const float*>(p.router_w);  // >= E + 1 floats, any values
+    fused_route_row(dc, p.ctrl + kStatus, 0, R, true);
+  }
 
   // ---- B: shared expert gate + up (no routing needed) ----------------------------------------
   if (p.has_shared) {
@@ -311,38 +385,77 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
   // ---- C: routing + grouping (every CTA, in its own shared memory) ---------------------------
   bar.wait(1);
   MOE_STAMP(5);
-  if (warp < m) fused_route_row(p, warp, R);
+  if (warp < m) fused_route_row(route_cfg(p), p.ctrl + kStatus, warp, R, false);
+  MOE_STAMP(12);
   __syncthreads();
-  fused_group(p, R);
+  fused_group(te, R);
+  if (tid == 0) {  // thread 0 wrote n_active in fused_group
+    const int n_slots = R.n_active + p.has_shared;
+    const int n_tile = ncols > 0 ? min(n_slots, fp.tile_slots) : 0;
+    s_tile_mask = 0;
+    s_tile_n = n_tile;
+    if (n_tile > 0) mbar_init(&s_tile_bar, (unsigned)n_tile);
+  }
   __syncthreads();
   const int U = R.n_active;
   MOE_STAMP(6);
 
-  // ---- D: routed gate + up; this CTA's phase-E down rows into L2 ------------------------------
-  {
+  // ---- D: routed gate + up; this CTA's phase-E down rows on their way ------------------------
+  // The last warp takes the phase-E slots (active experts in slot order, then the shared
+  // expert), lane s slot s, s + 32: the first tile_slots slots are bulk-copied into this CTA's
+  // shared-memory tile (when their addresses allow), the others are asked into L2 (when the
+  // whole call's down rows fit comfortably there). Both arrive while gate/up streams. Issuing
+  // bulk copies can hold the issuing warp until earlier ones drain, so with a tile the last warp
+  // does only this and the gate/up rows go to the other warps.
+  const bool tile_call = s_tile_n > 0;
+  const int n_gu_warps = tile_call ? kFusedWarps - 1 : kFusedWarps;
+  if (warp == kFusedWarps - 1 && ncols > 0) {
     const size_t down_bytes =
         ((size_t)U * packed_row_bytes(FMT, p.I) + (p.has_shared ? packed_row_bytes(FMT, p.S) : 0)) *
         (size_t)h;
-    if (down_bytes <= (size_t)fp.l2_prefetch_cap && ncols > 0 && tid < U + p.has_shared) {
-      const bool sh = tid == U;
-      const MatDev& D = sh ? p.sd : p.rd;
-      const int e = sh ? 0 : R.slot_e[tid];
-      const size_t rbytes = packed_row_bytes(FMT, D.k);
-      prefetch_l2_bulk(D.packed + (size_t)e * D.estride + (size_t)c0 * rbytes, ncols * rbytes);
-      if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) {
-        const size_t sb = (size_t)(D.k / 64) * 2;
-        prefetch_l2_lines(D.scales + (size_t)e * D.sstride + (size_t)c0 * sb, ncols * sb);
-        prefetch_l2_lines(D.biases + (size_t)e * D.sstride + (size_t)c0 * sb, ncols * sb);
-      } else if constexpr (FMT == MOE_FMT_NVFP4) {
-        const size_t sb = (size_t)(D.k / 16);
-        prefetch_l2_lines(D.scales + (size_t)e * D.sstride + (size_t)c0 * sb, ncols * sb);
+    for (int sl = lane; sl < U + p.has_shared; sl += 32) {
+      const bool sh = sl == U;
+      const MatDev D = pick_mat(sh, p.sd, p.rd);
+      const int e = sh ? 0 : R.slot_e[sl];
+      const int K = sh ? p.S : p.I;
+      const size_t prb = packed_row_bytes(FMT, K);
+      const size_t srb = FMT == MOE_FMT_Q4_AFFINE_G64 ? (size_t)(K / 64) * 2
+                         : FMT == MOE_FMT_NVFP4        ? (size_t)(K / 16)
+                                                       : 0;
+      const uint8_t* wsrc = D.packed + (size_t)e * D.estride + (size_t)c0 * prb;
+      const uint8_t* ssrc = srb ? D.scales + (size_t)e * D.sstride + (size_t)c0 * srb : nullptr;
+      const uint8_t* bsrc = FMT == MOE_FMT_Q4_AFFINE_G64
+                                ? D.biases + (size_t)e * D.sstride + (size_t)c0 * srb
+                                : nullptr;
+      const unsigned wb = (unsigned)(ncols * prb), sb = (unsigned)(ncols * srb);
+      if (FMT == MOE_FMT_NVFP4) R.ts[sl] = __ldg(D.tscale + e);
+      bool in_tile = false;
+      if (sl < s_tile_n) {
+        in_tile = sb % 16 == 0 && ((uintptr_t)ssrc | (uintptr_t)bsrc) % 16 == 0;
+        if (in_tile) {
+          uint8_t* dst = fsmem + fp.tile_off + (size_t)sl * fp.tile_slot_bytes;
+          const unsigned tx = wb + (FMT == MOE_FMT_Q4_AFFINE_G64 ? 2 * sb : sb);
+          mbar_arrive_expect_tx(&s_tile_bar, tx);
+          bulk_g2s(dst, wsrc, wb, &s_tile_bar);
+          if (srb) bulk_g2s(dst + fp.tile_sc_off, ssrc, sb, &s_tile_bar);
+          if (FMT == MOE_FMT_Q4_AFFINE_G64) bulk_g2s(dst + fp.tile_bi_off, bsrc, sb, &s_tile_bar);
+          atomicOr(&s_tile_mask, 1ull << sl);
+        } else {
+          mbar_arrive(&s_tile_bar);
+        }
+      }
+      if (!in_tile && down_bytes <= (size_t)fp.l2_prefetch_cap) {
+        prefetch_l2_bulk(wsrc, wb);
+        if (srb) prefetch_l2_lines(ssrc, sb);
+        if (bsrc) prefetch_l2_lines(bsrc, sb);
       }
     }
   }
+  MOE_STAMP(17);
   {
     const long long UI = (long long)U * p.I;
     const long long q0 = (long long)cta * UI / G, q1 = (long long)(cta + 1) * UI / G;
-    for (long long q = q0 + warp; q < q1; q += kFusedWarps) {
+    for (long long q = q0 + warp; warp < n_gu_warps && q < q1; q += n_gu_warps) {
       const int a = (int)(q / p.I), i = (int)(q - (long long)a * p.I);
       const int e = R.slot_e[a], beg = R.slot_beg[a], n = R.slot_n[a];
       const float* xr[RB];
@@ -398,15 +511,24 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
   }
   __syncthreads();
   MOE_STAMP(9);
-  {
-    // units: column pairs of each slot (the routed slots, then the shared expert)
+  const unsigned long long tile_mask = s_tile_mask;
+  if (tile_mask && !mbar_wait_bounded(&s_tile_bar, 0, fp.spin_limit)) {
+    atomicExch(p.ctrl + kStatus, (unsigned)MOE_ERR_DEVICE_TIMEOUT);
+    mbar_wait_bounded(&s_tile_bar, 0, fp.spin_limit);  // its copies still target this CTA
+  }
+  MOE_STAMP_AFTER(16, (unsigned)tile_mask);
+  // units: column pairs of each slot (the routed slots, then the shared expert). A CTA with a
+  // down-row tile reads every row through plain loads (tile slots from shared memory, the rest
+  // from L2); one without streams its rows from global memory. Same arithmetic either way.
+  auto down_units = [&](auto plain_tag) {
+    constexpr bool kPlain = decltype(plain_tag)::value;
     const int npair = (ncols + 1) / 2;
     const int n_units = npair * (U + p.has_shared);
     for (int u = warp; u < n_units; u += kFusedWarps) {
       const int slot = u / npair, col = c0 + 2 * (u - slot * npair);
       const bool two = col + 1 < c0 + ncols;
       const bool sh = slot == U;
-      const MatDev& D = sh ? p.sd : p.rd;
+      const MatDev D = pick_mat(sh, p.sd, p.rd);
       const int e = sh ? 0 : R.slot_e[slot];
       const int beg = sh ? te : R.slot_beg[slot];
       const int n = sh ? m : R.slot_n[slot];
@@ -420,14 +542,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
         xsr[j] = actsum + (size_t)r * (ld / 32);
       }
       const int nch = (int)(packed_row_bytes(FMT, K) / 16);
-      const RowRef A = row_ref<FMT>(D, e, col);
+      const bool in_tile = kPlain && ((tile_mask >> slot) & 1ull);
+      const uint8_t* sl = fsmem + fp.tile_off + (size_t)slot * fp.tile_slot_bytes;
+      RowRef A = in_tile ? tile_row_ref<FMT>(D, e, sl, K, fp, col - c0)
+                         : row_ref<FMT>(D, e, col);
+      if (FMT == MOE_FMT_NVFP4) A.ts = R.ts[slot];
       float a0[RB], a1[RB];
-      if (two) {
-        const RowRef B = row_ref<FMT>(D, e, col + 1);
-        rows2_dot<FMT, RB, false>(A, B, nch, xr, xsr, n, a0, a1);
-      } else {
-        rows1_dot<FMT, RB, false>(A, nch, xr, xsr, n, a0);
-      }
+      // an odd last column pairs with itself (one code path; its second result is dropped)
+      const int col_b = two ? col + 1 : col;
+      const RowRef B = in_tile ? tile_row_ref<FMT>(D, e, sl, K, fp, col_b - c0)
+                               : row_ref<FMT>(D, e, col_b);
+      rows2_dot<FMT, RB, kPlain>(A, B, nch, xr, xsr, n, a0, a1);
       if (lane < n) {
         float v0 = 0.f, v1 = 0.f;
 #pragma unroll
@@ -440,6 +565,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
         if (two) ys[(size_t)(beg + lane) * ncols + (col + 1 - c0)] = v1 * A.ts;
       }
     }
+  };
+  if (tile_mask) {
+    down_units(std::true_type{});
+  } else {
+    down_units(std::false_type{});
   }
   __syncthreads();
   MOE_STAMP(10);

@@ -75,81 +75,174 @@ __device__ __forceinline__ uint32_t key_bits(float v) {
 
 // Routing of row r by one warp. Lane s < k ends with the s-th selected expert (descending key,
 // ties to the lower id) and its weight; every lane gets gamma (shared-expert gate, or 1).
-// Each of the k rounds is a lane-local arg-max over the lane's 8 candidates followed by two
-// warp reductions (max key, then min id among lanes holding that key). Returns false when a
-// selected key is not a finite number.
-__device__ __forceinline__ bool route_row(const Params& p, int r, int& my_id, float& my_w,
-                                          float& gamma) {
+// `bias` holds the expert biases (global memory or a shared-memory copy), read only when the
+// keys are biased sigmoid scores. Every load of the row (logits, biases, the shared-gate logit)
+// is issued before the first one is used. Each lane then sorts its NJ = E/32 candidates once;
+// a selection round is one warp max over the lanes' heads and a ballot of the lanes holding it
+// (a second reduction, min id, only when several lanes tie), after which the winning lane pops
+// its head. Returns false when a selected key is not a finite number.
+// The routing options of a call, copied out of the kernel parameters into registers (a routine
+// that reads them through a reference to the parameter block would load each one from memory).
+struct RouteCfg {
+  const float* logits;  // [m, E + 1]
+  int E, k, routing, raw, has_bias, norm, gated;
+  float rsf;
+  unsigned long long* stamps;  // phase timestamps (timer builds only)
+};
+
+__device__ __forceinline__ RouteCfg route_cfg(const Params& p) {
+  RouteCfg c;
+  c.logits = p.logits;
+  c.E = p.E;
+  c.k = p.k;
+  c.routing = p.routing;
+  c.raw = p.raw;
+  c.has_bias = p.has_bias;
+  c.norm = p.norm;
+  c.gated = p.shared_kind == MOE_SHARED_SIGMOID_GATE;
+  c.rsf = p.rsf;
+  c.stamps = reinterpret_cast<unsigned long long*>(p.ypart);
+  return c;
+}
+
+#ifdef MOE_PHASE_TIMERS
+#define MOE_ROUTE_STAMP(slot, v)                                                            \
+  do {                                                                                      \
+    if (threadIdx.x == 0) {                                                                 \
+      unsigned long long t_;                                                                \
+      asm volatile("{ .reg .u32 d_; mov.u32 d_, %1; mov.u64 %0, %%clock64; }"               \
+                   : "=l"(t_) : "r"((unsigned)(v)) : "memory");                              \
+      c.stamps[blockIdx.x * kPhaseSlots + (slot)] = t_;                                      \
+    }                                                                                       \
+  } while (0)
+#else
+#define MOE_ROUTE_STAMP(slot, v) \
+  do {                           \
+  } while (0)
+#endif
+
+template <int NJ>
+__device__ __forceinline__ bool route_row_nj(const RouteCfg& c, int r, const float* bias,
+                                             int& my_id, float& my_w, float& gamma) {
+  constexpr unsigned kFull = 0xffffffffu;
   const int lane = threadIdx.x & 31;
-  const int E = p.E, k = p.k;
-  const float* lrow = p.logits + (size_t)r * (E + 1);
-  float lg[8];
-  uint32_t key[8];
+  const int E = c.E, k = c.k;
+  const float* lrow = c.logits + (size_t)r * (E + 1);
+  const bool sig_keys = c.routing == MOE_ROUTE_SIGMOID && !c.raw;
+  const bool add_bias = sig_keys && c.has_bias;
+  const bool gated = c.gated;
+  float lg[NJ], bs[NJ];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < NJ; ++j) {
     const int e = lane + 32 * j;
     lg[j] = e < E ? __ldcg(lrow + e) : -INFINITY;
+    bs[j] = (add_bias && e < E) ? bias[e] : 0.f;
   }
+  const float glog = gated ? __ldcg(lrow + E) : 0.f;
+  MOE_ROUTE_STAMP(13, __float_as_uint(lg[0]) ^ __float_as_uint(bs[0]) ^ __float_as_uint(glog));
+  uint32_t key[NJ];
+  int id[NJ];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < NJ; ++j) {
     const int e = lane + 32 * j;
     float kv = lg[j];
-    if (p.routing == MOE_ROUTE_SIGMOID && !p.raw) {
+    if (sig_keys) {
       kv = 1.0f / (1.0f + expf(-lg[j]));
-      if (p.has_bias && e < E) kv += __ldg(p.expert_bias + e);
+      if (add_bias) kv += bs[j];
     }
-    key[j] = e < E ? key_bits(kv) : 0u;
+    key[j] = e < E ? key_bits(kv) : 0u;  // a real key is >= key_bits(-inf) > 0
+    id[j] = e;
   }
-  float mx = -INFINITY, den = 0.f;
-  if (p.routing == MOE_ROUTE_SOFTMAX) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) mx = fmaxf(mx, lg[j]);
-    mx = warp_max(mx);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) den += (lane + 32 * j < E) ? expf(lg[j] - mx) : 0.f;
-    den = warp_sum(den);
+  // sort network: position a ends before position b (descending key, then ascending id)
+  auto cx = [&](int a, int b) {
+    if (key[b] > key[a] || (key[b] == key[a] && id[b] < id[a])) {
+      const uint32_t tk = key[a];
+      key[a] = key[b];
+      key[b] = tk;
+      const int ti = id[a];
+      id[a] = id[b];
+      id[b] = ti;
+      const float tl = lg[a];
+      lg[a] = lg[b];
+      lg[b] = tl;
+    }
+  };
+  if constexpr (NJ == 2) cx(0, 1);
+  if constexpr (NJ == 4) {
+    cx(0, 1); cx(2, 3); cx(0, 2); cx(1, 3); cx(1, 2);
   }
-  unsigned taken = 0;
+  if constexpr (NJ == 8) {
+    cx(0, 2); cx(1, 3); cx(4, 6); cx(5, 7); cx(0, 4); cx(1, 5); cx(2, 6); cx(3, 7);
+    cx(0, 1); cx(2, 3); cx(4, 5); cx(6, 7); cx(2, 4); cx(3, 5); cx(1, 4); cx(3, 6);
+    cx(1, 2); cx(3, 4); cx(5, 6);
+  }
+  MOE_ROUTE_STAMP(14, key[0] ^ (uint32_t)id[0] ^ __float_as_uint(lg[0]));
+  const bool softmax = c.routing == MOE_ROUTE_SOFTMAX;
   bool ok = true;
   my_id = 0;
-  float my_l = 0.f;
-  for (int s = 0; s < k; ++s) {
-    uint32_t bk = 0;
-    int bj = -1;
+  float my_l = 0.f, top_l = 0.f, den = 0.f;
+#pragma unroll 1
+  for (int s = 0; s < k; ++s) {  // kept rolled: the body is fetched once, not k times
+    const uint32_t best = __reduce_max_sync(kFull, key[0]);
+    const bool mine = key[0] == best;
+    const unsigned tied = __ballot_sync(kFull, mine);
+    int owner = __ffs(tied) - 1;
+    if (tied & (tied - 1u))
+      owner = (int)(__reduce_min_sync(kFull, mine ? (uint32_t)id[0] : 0xffffffffu) & 31u);
+    const int sid = __shfl_sync(kFull, id[0], owner);
+    const float sl = __shfl_sync(kFull, lg[0], owner);
+    if (best <= key_bits(-INFINITY)) ok = false;  // -inf or NaN won a slot
+    if (s == 0) {
+      top_l = sl;  // softmax keys are the logits: the first winner holds the largest one
+      if (softmax && !c.norm) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {  // ascending ids within the lane: strict > keeps the lowest
-      if (!((taken >> j) & 1u) && lane + 32 * j < E && (bj < 0 || key[j] > bk)) {
-        bk = key[j];
-        bj = j;
+        for (int j = 0; j < NJ; ++j) den += expf(lg[j] - top_l);  // -inf past E adds 0
       }
     }
-    const uint32_t best = __reduce_max_sync(0xffffffffu, bj >= 0 ? bk : 0u);
-    const uint32_t cand = (bj >= 0 && bk == best) ? (uint32_t)(lane + 32 * bj) : 0xFFFFFFFFu;
-    const uint32_t id = __reduce_min_sync(0xffffffffu, cand);
-    const int owner = (int)(id & 31u);
-    float l = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (lane == owner && (int)(id >> 5) == j) l = lg[j];
-    l = __shfl_sync(0xffffffffu, l, owner);
-    if (lane == owner) taken |= 1u << (id >> 5);
-    if (best <= key_bits(-INFINITY)) ok = false;  // -inf or NaN won a slot
     if (lane == s) {
-      my_id = (int)id;
-      my_l = l;
+      my_id = sid;
+      my_l = sl;
+    }
+    if (lane == owner) {
+#pragma unroll
+      for (int j = 0; j + 1 < NJ; ++j) {
+        key[j] = key[j + 1];
+        id[j] = id[j + 1];
+        lg[j] = lg[j + 1];
+      }
+      key[NJ - 1] = 0u;
+      id[NJ - 1] = 0x7fffffff;
+      lg[NJ - 1] = -INFINITY;
     }
   }
-  float wv = 0.f;
-  if (lane < k)
-    wv = (p.routing == MOE_ROUTE_SOFTMAX) ? expf(my_l - mx) / den : 1.0f / (1.0f + expf(-my_l));
-  if (p.norm) {
-    const float tot = warp_sum(lane < k ? wv : 0.f);
+  MOE_ROUTE_STAMP(15, (uint32_t)my_id ^ __float_as_uint(my_l) ^ __float_as_uint(top_l));
+  float wv;
+  if (softmax) {
+    // exp(l - max) / sum over all experts; under renormalisation the full sum cancels
+    wv = expf(my_l - top_l);
+    if (!c.norm) wv = wv / warp_sum(den);
+  } else {
+    wv = 1.0f / (1.0f + expf(-my_l));
+  }
+  if (lane >= k) wv = 0.f;
+  if (c.norm) {
+    // lanes >= k hold 0, so the k-lane sum needs only the xor steps below the next power of 2
+    float tot = wv;
+    for (int off = (k > 4 ? 4 : k > 2 ? 2 : k > 1 ? 1 : 0); off > 0; off >>= 1)
+      tot += __shfl_xor_sync(kFull, tot, off);
     wv = wv / tot;
   }
-  my_w = wv * p.rsf;
-  gamma = 1.f;
-  if (p.shared_kind == MOE_SHARED_SIGMOID_GATE) gamma = 1.0f / (1.0f + expf(-__ldcg(lrow + E)));
+  my_w = wv * c.rsf;
+  gamma = gated ? 1.0f / (1.0f + expf(-glog)) : 1.f;
   return ok;
+}
+
+__device__ __forceinline__ bool route_row(const RouteCfg& c, int r, const float* bias, int& my_id,
+                                          float& my_w, float& gamma) {
+  if (c.E <= 32) return route_row_nj<1>(c, r, bias, my_id, my_w, gamma);
+  if (c.E <= 64) return route_row_nj<2>(c, r, bias, my_id, my_w, gamma);
+  if (c.E <= 128) return route_row_nj<4>(c, r, bias, my_id, my_w, gamma);
+  return route_row_nj<8>(c, r, bias, my_id, my_w, gamma);
 }
 
 // Routing of row r for the multi-kernel path: route_row, then the global and shared writes.
@@ -157,7 +250,7 @@ __device__ void route_row_warp(const Params& p, int r, int* s_idx) {
   const int lane = threadIdx.x & 31;
   int id;
   float w, g;
-  const bool ok = route_row(p, r, id, w, g);
+  const bool ok = route_row(route_cfg(p), r, p.expert_bias, id, w, g);
   if (lane < p.k) {
     p.idx[r * p.k + lane] = id;
     p.wts[r * p.k + lane] = w;

@@ -193,6 +193,11 @@ class DeviceLayer:
         B.moe_decode_forward(self.c, m, x, self.router_w, self.expert_bias, self.routed,
                              self.shared, self.shared_gate_w, out, ws, ws.numel(), st)
 
+    def launches(self, m: int) -> int:
+        """Kernel launches one forward call with m rows makes on this device."""
+        with torch.cuda.device(self.device):
+            return B.moe_decode_launches(self.c, m, self.routed, self.shared)
+
     def read_routing(self, m: int, ws: torch.Tensor, stream=None):
         st = stream if stream is not None else torch.cuda.current_stream(self.device)
         return B.moe_decode_read_routing(self.c, m, ws, ws.numel(), st)

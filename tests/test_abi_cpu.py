@@ -126,6 +126,27 @@ def test_valid_call_without_gpu_reports_cuda_or_device_error():
     assert rc in (B.MOE_ERR_CUDA, B.MOE_ERR_UNSUPPORTED_DEVICE)
 
 
+def _launches(c, m=1, routed=None, shared=None, out=True):
+    n = ctypes.c_int32(-1)
+    routed = routed if routed is not None else _fake_table()
+    return B.lib.moe_decode_launches(ctypes.byref(c), m, ctypes.byref(routed),
+                                     ctypes.byref(shared) if shared is not None else None,
+                                     ctypes.byref(n) if out else None)
+
+
+def test_launch_count_query_refusals():
+    c = _small_cfg()
+    assert _launches(c, m=0) == B.MOE_ERR_BAD_SHAPE
+    assert _launches(c, out=False) == B.MOE_ERR_NULL_POINTER
+    t = _fake_table()
+    t.up.format = B.MOE_FMT_NVFP4
+    assert _launches(c, routed=t) == B.MOE_ERR_BAD_FORMAT
+    c5 = _small_cfg(shared_inter=64, shared_kind="plain")
+    assert _launches(c5) == B.MOE_ERR_NULL_POINTER       # shared table required
+    if not torch.cuda.is_available():
+        assert _launches(c) in (B.MOE_ERR_CUDA, B.MOE_ERR_UNSUPPORTED_DEVICE)
+
+
 # ---- pack / quantise helpers ---------------------------------------------------------------
 
 def test_packed_bytes():

@@ -241,3 +241,11 @@ def test_persistent_kernel_and_chain_agree_bitwise(name, m):
     rows = SAMPLE_ROWS.get((name, m))
     want, _ = ref.moe_forward(olay, x, rows=rows)
     check_out(auto if rows is None else auto[rows], want)
+
+
+def test_launch_count_follows_the_dispatch_rule():
+    lay, dev, _ = layer_for(CONFIGS["qwen3_30b_a3b"])
+    assert [dev.launches(m) for m in (1, 2, 3, 4)] == [1, 1, 1, 1]
+    assert [dev.launches(m) for m in (5, 8, 64)] == [3, 3, 3]
+    with _Path("chain"):
+        assert dev.launches(1) == 3
