@@ -163,6 +163,16 @@ int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, const void* rou
 int moe_decode_launches(const moe_cfg* cfg, int m, const moe_expert_table* routed,
                         const moe_expert_table* shared, int* launches);
 
+/* Test aid for failure detection without a GPU fault. After this call the persistent kernel's
+ * grid-barrier waits expect `extra_arrivals` (0 or 1) more arrivals than any launch makes and
+ * give up after `spin_limit_cycles` SM clock cycles (0: the default budget of about a second).
+ * Every wait stays bounded, so each launch ends; its workspace status then reads
+ * MOE_ERR_DEVICE_TIMEOUT and its outputs are undefined (call moe_workspace_init before reusing
+ * the workspace). moe_debug_barrier_test(0, 0) restores normal operation. Process-wide; do not
+ * call it while other threads run forward calls. Returns MOE_ERR_BAD_OPTION for other values.
+ * The decode pages have no counterpart. */
+int moe_debug_barrier_test(int extra_arrivals, long long spin_limit_cycles);
+
 /* Copy the routing and grouping of the last forward call that used `workspace` to host arrays
  * (synchronises `stream`). Any output pointer may be NULL to skip it. Sizes: idx, weights,
  * sorted_pairs, token_to_perm: m*top_k; expert_offsets: num_experts+1; active: min(m*top_k, E);

@@ -49,6 +49,7 @@ EXPORTS = (
     "moe_get_device_status", "moe_packed_bytes", "moe_pack_bf16", "moe_quantize_q4_affine",
     "moe_quantize_nvfp4", "moe_dequantize", "moe_status_string", "moe_last_cuda_error",
     "moe_version", "moe_decode_forward_no_alloc", "moe_decode_launches",
+    "moe_debug_barrier_test",
 )
 
 MOE_NO_ALLOC_SCRATCH_BYTES = 16 << 20
@@ -112,6 +113,7 @@ def _load() -> ctypes.CDLL:
                                         P(moe_expert_table), vp, vp, vp],
         "moe_decode_launches": [P(moe_cfg), i32, P(moe_expert_table), P(moe_expert_table),
                                 P(ctypes.c_int32)],
+        "moe_debug_barrier_test": [i32, i64],
         "moe_status_string": [i32],
         "moe_last_cuda_error": [],
         "moe_version": [],
@@ -198,6 +200,11 @@ def moe_decode_launches(cfg: moe_cfg, m: int, routed: moe_expert_table,
                                  ctypes.byref(n))
     _check(rc, "moe_decode_launches")
     return int(n.value)
+
+
+def moe_debug_barrier_test(extra_arrivals: int, spin_limit_cycles: int) -> None:
+    """Failure-detection test aid: make the persistent kernel's grid-barrier waits run out."""
+    _check(lib.moe_debug_barrier_test(extra_arrivals, spin_limit_cycles), "moe_debug_barrier_test")
 
 
 def moe_decode_read_routing(cfg: moe_cfg, m: int, workspace, workspace_bytes: int, stream=None):

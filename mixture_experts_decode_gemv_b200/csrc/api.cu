@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include <cstdlib>
@@ -233,6 +234,11 @@ int forced_path() {
 }
 
 size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
+
+constexpr long long kSpinLimit = 2000000000LL;  // about a second of SM clock cycles
+// Failure-detection test settings (moe_debug_barrier_test); zero in normal use.
+std::atomic<int> g_test_bar_extra{0};
+std::atomic<long long> g_test_spin_limit{0};
 constexpr size_t kFusedSmemBudget = 220 * 1024;
 
 // Shared-memory plan of the persistent kernel; false when the layer does not fit it.
@@ -277,7 +283,9 @@ bool plan_fused(const moe_cfg& c, int m, bool has_shared, int fmt, int sms, Fuse
   fp->cols_per_cta = cols;
   fp->act_ld = ld;
   fp->smem_bytes = (int)off;
-  fp->spin_limit = 2000000000LL;  // about a second of clock cycles
+  fp->spin_limit = g_test_spin_limit.load() > 0 ? g_test_spin_limit.load() : kSpinLimit;
+  fp->tile_limit = kSpinLimit;
+  fp->bar_extra = (unsigned)g_test_bar_extra.load();
   fp->l2_prefetch_cap = 48LL << 20;
   return true;
 }
@@ -528,6 +536,13 @@ extern "C" int moe_decode_launches(const moe_cfg* cfg, int m, const moe_expert_t
   FusedPlan fp;
   *launches = use_fused(*cfg, m, routed, shared, has_shared, &fp)
                   ? 1 : chain_launches(routed, shared, has_shared);
+  return MOE_OK;
+}
+
+extern "C" int moe_debug_barrier_test(int extra_arrivals, long long spin_limit_cycles) {
+  if (extra_arrivals < 0 || extra_arrivals > 1 || spin_limit_cycles < 0) return MOE_ERR_BAD_OPTION;
+  g_test_spin_limit.store(spin_limit_cycles);
+  g_test_bar_extra.store(extra_arrivals);
   return MOE_OK;
 }
 

@@ -341,6 +341,58 @@ __device__ __forceinline__ void rows2_dot(const RowRef& A, const RowRef& B, int 
   }
 }
 
+// NR weight rows (same length, nch chunks) against nb <= RB activation rows: rows2_dot for any
+// number of rows, with the same per-row arithmetic (chunk order per lane, then a butterfly
+// sum), so every row's bits match rows2_dot's. With plain loads from shared memory, one chunk
+// per row and lane is in flight (NR >= 4) and the activations are re-read per row from shared
+// memory; acc[r][j] receives the full dot product of row r with activation row j.
+template <int FMT, int RB, bool PLAIN, int NR>
+__device__ __forceinline__ void rowsN_dot(const RowRef (&A)[NR], int nch,
+                                          const float* const (&xr)[RB],
+                                          const float* const (&xsr)[RB], int nb,
+                                          float (&acc)[NR][RB]) {
+  constexpr int U = PLAIN ? (NR >= 4 ? 1 : 2) : row_unroll<FMT, false, RB>();
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int r = 0; r < NR; ++r)
+#pragma unroll
+    for (int j = 0; j < RB; ++j) acc[r][j] = 0.f;
+  for (int c0 = lane; c0 < nch; c0 += 32 * U) {
+    Chunk ch[U][NR];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nch) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) ch[u][r] = load_chunk<FMT, PLAIN>(A[r], c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < nch) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          Dec<FMT> d;
+          decode<FMT>(ch[u][r], d);
+#pragma unroll
+          for (int j = 0; j < RB; ++j) {
+            if (j < nb) {
+              float sx = 0.f;
+              if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64) sx = xsr[j][c];
+              acc[r][j] += dot<FMT>(d, xr[j], c, sx);
+            }
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < NR; ++r)
+#pragma unroll
+    for (int j = 0; j < RB; ++j) acc[r][j] = warp_allsum(acc[r][j]);
+}
+
 // One weight row (same arithmetic per row as rows2_dot).
 template <int FMT, int RB, bool SMEM>
 __device__ __forceinline__ void rows1_dot(const RowRef& A, int nch,

@@ -48,8 +48,10 @@ struct FusedPlan {
   int tile_sc_off;    // within a slot: scales rows, then (Q4) biases rows at 2 * tile_sc_off -
   int tile_bi_off;    //   packed rows first, each block 16-byte aligned
   int smem_bytes;
-  long long spin_limit;       // clock cycles a barrier wait may spin before it gives up
+  long long spin_limit;       // clock cycles a grid-barrier wait may spin before it gives up
+  long long tile_limit;       // the same for the down-row tile's copies
   long long l2_prefetch_cap;  // largest per-call down-projection byte count asked into L2
+  unsigned bar_extra;         // arrivals a barrier waits for beyond the grid (0; 1 in tests)
 };
 
 
@@ -139,6 +141,7 @@ struct GridBarrier {
   unsigned* status;
   unsigned long long base;
   long long limit;
+  unsigned extra;  // 0, or 1 to make every wait run out (failure-detection tests)
 
   __device__ void arrive() const {
     __syncthreads();
@@ -147,7 +150,7 @@ struct GridBarrier {
   }
   __device__ void wait(unsigned passed) const {
     if (threadIdx.x == 0) {
-      const unsigned long long target = base + (unsigned long long)passed * gridDim.x;
+      const unsigned long long target = base + (unsigned long long)passed * gridDim.x + extra;
       const long long t0 = clock64();
       unsigned long long seen;
       while ((seen = ld_acquire_u64(ctr)) < target) {
@@ -324,7 +327,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
     return (const uint8_t*)p.x + (size_t)j * xrow_bytes;
   }, 0, kFusedThreads);
   __syncthreads();
-  const GridBarrier bar{bar_ctr, p.ctrl + kStatus, s_base, fp.spin_limit};
+  const GridBarrier bar{bar_ctr, p.ctrl + kStatus, s_base, fp.spin_limit, fp.bar_extra};
   MOE_STAMP(2);
 
   // ---- A: router logits, one warp per (router row, activation row) ----------------------------
@@ -352,6 +355,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
     RouteCfg dc = route_cfg(p);
     dc.logits = reinterpret_cast<const float*>(p.router_w);  // >= E + 1 floats, any values
     fused_route_row(dc, p.ctrl + kStatus, 0, R, true);
+#ifdef MOE_PHASE_TIMERS
+    if (lane == 0) {
+      unsigned long long t_;
+      asm volatile("mov.u64 %0, %%clock64;" : "=l"(t_)::"memory");
+      reinterpret_cast<unsigned long long*>(p.ypart)[blockIdx.x * kPhaseSlots + 18] = t_;
+    }
+#endif
   }
 
   // ---- B: shared expert gate + up (no routing needed) ----------------------------------------
@@ -451,7 +461,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
       }
     }
   }
-  MOE_STAMP(17);
   {
     const long long UI = (long long)U * p.I;
     const long long q0 = (long long)cta * UI / G, q1 = (long long)(cta + 1) * UI / G;
@@ -512,9 +521,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
   __syncthreads();
   MOE_STAMP(9);
   const unsigned long long tile_mask = s_tile_mask;
-  if (tile_mask && !mbar_wait_bounded(&s_tile_bar, 0, fp.spin_limit)) {
+  if (tile_mask && !mbar_wait_bounded(&s_tile_bar, 0, fp.tile_limit)) {
     atomicExch(p.ctrl + kStatus, (unsigned)MOE_ERR_DEVICE_TIMEOUT);
-    mbar_wait_bounded(&s_tile_bar, 0, fp.spin_limit);  // its copies still target this CTA
+    mbar_wait_bounded(&s_tile_bar, 0, fp.tile_limit);  // its copies still target this CTA
   }
   MOE_STAMP_AFTER(16, (unsigned)tile_mask);
   // units: column pairs of each slot (the routed slots, then the shared expert). A CTA with a
@@ -522,11 +531,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
   // from L2); one without streams its rows from global memory. Same arithmetic either way.
   auto down_units = [&](auto plain_tag) {
     constexpr bool kPlain = decltype(plain_tag)::value;
-    const int npair = (ncols + 1) / 2;
-    const int n_units = npair * (U + p.has_shared);
+    constexpr int NR = kPlain ? 4 : 2;  // output columns per unit
+    const int nblk = (ncols + NR - 1) / NR;
+    const int n_units = nblk * (U + p.has_shared);
     for (int u = warp; u < n_units; u += kFusedWarps) {
-      const int slot = u / npair, col = c0 + 2 * (u - slot * npair);
-      const bool two = col + 1 < c0 + ncols;
+      const int slot = u / nblk, col = c0 + NR * (u - slot * nblk);
+      const int nvalid = min(NR, c0 + ncols - col);
       const bool sh = slot == U;
       const MatDev D = pick_mat(sh, p.sd, p.rd);
       const int e = sh ? 0 : R.slot_e[slot];
@@ -544,26 +554,27 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
       const int nch = (int)(packed_row_bytes(FMT, K) / 16);
       const bool in_tile = kPlain && ((tile_mask >> slot) & 1ull);
       const uint8_t* sl = fsmem + fp.tile_off + (size_t)slot * fp.tile_slot_bytes;
-      RowRef A = in_tile ? tile_row_ref<FMT>(D, e, sl, K, fp, col - c0)
-                         : row_ref<FMT>(D, e, col);
-      if (FMT == MOE_FMT_NVFP4) A.ts = R.ts[slot];
-      float a0[RB], a1[RB];
-      // an odd last column pairs with itself (one code path; its second result is dropped)
-      const int col_b = two ? col + 1 : col;
-      const RowRef B = in_tile ? tile_row_ref<FMT>(D, e, sl, K, fp, col_b - c0)
-                               : row_ref<FMT>(D, e, col_b);
-      rows2_dot<FMT, RB, kPlain>(A, B, nch, xr, xsr, n, a0, a1);
-      if (lane < n) {
-        float v0 = 0.f, v1 = 0.f;
+      // columns past the CTA's last repeat its last column (results dropped)
+      RowRef A[NR];
 #pragma unroll
-        for (int j = 0; j < RB; ++j)
-          if (j == lane) {
-            v0 = a0[j];
-            if (two) v1 = a1[j];
-          }
-        ys[(size_t)(beg + lane) * ncols + (col - c0)] = v0 * A.ts;
-        if (two) ys[(size_t)(beg + lane) * ncols + (col + 1 - c0)] = v1 * A.ts;
+      for (int r = 0; r < NR; ++r) {
+        const int cr = col + min(r, nvalid - 1);
+        A[r] = in_tile ? tile_row_ref<FMT>(D, e, sl, K, fp, cr - c0) : row_ref<FMT>(D, e, cr);
       }
+      const float ts = FMT == MOE_FMT_NVFP4 ? R.ts[slot] : 1.f;
+      float acc[NR][RB];
+      rowsN_dot<FMT, RB, kPlain, NR>(A, nch, xr, xsr, n, acc);
+      if (lane < n) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          float v = 0.f;
+#pragma unroll
+          for (int j = 0; j < RB; ++j)
+            if (j == lane) v = acc[r][j];
+          if (r < nvalid) ys[(size_t)(beg + lane) * ncols + (col + r - c0)] = v * ts;
+        }
+      }
+      if (u == warp) MOE_STAMP_AFTER(17, __float_as_uint(acc[0][0]));  // warp 0's first unit
     }
   };
   if (tile_mask) {

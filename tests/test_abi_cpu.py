@@ -147,6 +147,13 @@ def test_launch_count_query_refusals():
         assert _launches(c) in (B.MOE_ERR_CUDA, B.MOE_ERR_UNSUPPORTED_DEVICE)
 
 
+def test_barrier_test_hook_validates_its_arguments():
+    assert B.lib.moe_debug_barrier_test(2, 0) == B.MOE_ERR_BAD_OPTION
+    assert B.lib.moe_debug_barrier_test(-1, 0) == B.MOE_ERR_BAD_OPTION
+    assert B.lib.moe_debug_barrier_test(0, -5) == B.MOE_ERR_BAD_OPTION
+    assert B.lib.moe_debug_barrier_test(0, 0) == B.MOE_OK
+
+
 # ---- pack / quantise helpers ---------------------------------------------------------------
 
 def test_packed_bytes():

@@ -249,3 +249,30 @@ def test_launch_count_follows_the_dispatch_rule():
     assert [dev.launches(m) for m in (5, 8, 64)] == [3, 3, 3]
     with _Path("chain"):
         assert dev.launches(1) == 3
+
+
+def test_grid_barrier_timeout_is_reported_and_the_workspace_recovers():
+    """A barrier wait that runs out (made to expect one arrival too many, with a ~1 ms budget)
+    ends the launch with MOE_ERR_DEVICE_TIMEOUT in the workspace status; after
+    moe_workspace_init the same workspace gives the normal result again."""
+    lay, dev, _ = layer_for(CONFIGS["qwen3_30b_a3b"])
+    m = 1
+    assert dev.launches(m) == 1
+    x = dev.x_to_device(lay.x(m))
+    ws = dev.new_workspace(m)
+    want, out = dev.new_out(m), dev.new_out(m)
+    dev.forward(x, want, ws)
+    torch.cuda.synchronize()
+    assert dev.device_status(ws) == B.MOE_OK
+    B.moe_debug_barrier_test(1, 2_000_000)
+    try:
+        dev.forward(x, out, ws)
+        torch.cuda.synchronize()
+    finally:
+        B.moe_debug_barrier_test(0, 0)
+    assert dev.device_status(ws) == B.MOE_ERR_DEVICE_TIMEOUT
+    B.moe_workspace_init(ws, ws.numel(), torch.cuda.current_stream())
+    dev.forward(x, out, ws)
+    torch.cuda.synchronize()
+    assert dev.device_status(ws) == B.MOE_OK
+    assert torch.equal(out, want)
