@@ -42,7 +42,10 @@ Weight formats decoded here (storage defined by the library's pack helpers; 4-bi
  * 4-bit affine, group 64: ``w = scale * q + bias`` with fp16 scale and bias per 64 elements;
  * NVFP4: E2M1 codes, one E4M3 scale per 16 elements (the NVFP4 scale block of metrale
    ``helpers_a.rs``), one fp32 tensor scale per matrix (its ``weight_scale_2``):
-   ``w = e2m1(q) * e4m3(s) * tensor_scale``.
+   ``w = e2m1(q) * e4m3(s) * tensor_scale``;
+ * MXFP4: E2M1 codes, one E8M0 scale per 32 elements (the native MXFP4 scale block of metrale
+   ``helpers_a.rs``, the scale-block note of ``transpose_for_prefill_impl``), no tensor scale:
+   ``w = e2m1(q) * 2**(s - 127)`` (E8M0 as the OCP Microscaling specification defines it).
 Element 2j of a 4-bit row is the low nibble of byte j.
 
 Every function here is pinned by a CPU test against the pages' worked example, closed forms,
@@ -97,6 +100,12 @@ def e4m3_value(code: np.ndarray) -> np.ndarray:
     return np.where(s == 1, -mag, mag)
 
 
+def e8m0_value(code: np.ndarray) -> np.ndarray:
+    """E8M0 scale code -> value: an unsigned biased exponent, 2**(code - 127); 0xFF is NaN."""
+    c = np.asarray(code, dtype=np.int64)
+    return np.where(c == 255, np.nan, np.exp2(c - 127.0))
+
+
 def unpack_nibbles(packed: np.ndarray, k: int) -> np.ndarray:
     """``[n, k/2]`` bytes -> ``[n, k]`` 4-bit codes; element 2j is the low nibble of byte j."""
     p = np.asarray(packed, dtype=np.uint8)
@@ -127,6 +136,9 @@ def decode_matrix(slab, e: int = 0) -> np.ndarray:
         v = e2m1_value(unpack_nibbles(slab.data[e], k))
         blk = np.repeat(e4m3_value(slab.scales[e]), 16, axis=1)
         return v * blk * float(np.float32(slab.tensor_scale[e]))
+    if slab.fmt == "mxfp4":
+        v = e2m1_value(unpack_nibbles(slab.data[e], k))
+        return v * np.repeat(e8m0_value(slab.scales[e]), 32, axis=1)
     raise ValueError(f"unknown format {slab.fmt!r}")
 
 

@@ -119,3 +119,41 @@ def test_nvfp4_every_code_times_scale():
     e2m1 = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6])
     np.testing.assert_array_equal(w[:16], e2m1 * 2.0 ** -9)
     np.testing.assert_array_equal(w[16:], e2m1 * 448.0)
+
+
+def test_e8m0_golden_codes(golden_dir):
+    codes, vals = _read_table(os.path.join(golden_dir, "e8m0_values.txt"))
+    got = ref.e8m0_value(codes)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(vals))
+    np.testing.assert_array_equal(got[~np.isnan(vals)], vals[~np.isnan(vals)])
+
+
+def test_e8m0_every_code_is_a_power_of_two():
+    c = np.arange(255)
+    v = ref.e8m0_value(c)
+    m, ex = np.frexp(v)                       # v = m * 2**ex with m in [0.5, 1)
+    np.testing.assert_array_equal(m, 0.5)
+    np.testing.assert_array_equal(ex - 1, c - 127)
+
+
+def test_mxfp4_hand_built():
+    # 64 codes in two 32-element blocks: block 0 all code 5 (3.0), block 1 all code 0xA (-1.0)
+    q = np.array([5] * 32 + [0xA] * 32, dtype=np.uint8)
+    packed = (q[0::2] | (q[1::2] << 4)).astype(np.uint8)[None, None, :]
+    scales = np.array([[[0x7F, 0x81]]], dtype=np.uint8)          # 1.0, 4.0
+    slab = MatrixSlab("mxfp4", 1, 64, packed, scales=scales)
+    w = ref.decode_matrix(slab, 0)[0]
+    np.testing.assert_array_equal(w[:32], 3.0)
+    np.testing.assert_array_equal(w[32:], -4.0)
+
+
+def test_mxfp4_with_unit_scales_is_plain_e2m1_and_scales_by_powers_of_two():
+    rng = np.random.default_rng(3)
+    q = rng.integers(0, 16, size=(3, 96), dtype=np.uint8)
+    packed = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)[None]
+    sc = rng.integers(100, 150, size=(1, 3, 3), dtype=np.uint8)
+    w = ref.decode_matrix(MatrixSlab("mxfp4", 3, 96, packed, scales=sc), 0)
+    plain = ref.decode_matrix(MatrixSlab("mxfp4", 3, 96, packed,
+                                         scales=np.full_like(sc, 0x7F)), 0)
+    np.testing.assert_array_equal(plain, ref.e2m1_value(q))
+    np.testing.assert_array_equal(w, plain * np.exp2(np.repeat(sc[0].astype(float) - 127, 32, 1)))
