@@ -67,9 +67,14 @@ typedef enum moe_format {
   MOE_FMT_Q4_AFFINE_G64 = 2, /* 4-bit codes [n, k/2] (element 2j = low nibble of byte j);
                                 fp16 scales [n, k/64] and fp16 biases [n, k/64];
                                 w = scale * q + bias */
-  MOE_FMT_NVFP4 = 3          /* E2M1 codes [n, k/2] (low nibble first); E4M3 block scales
+  MOE_FMT_NVFP4 = 3,         /* E2M1 codes [n, k/2] (low nibble first); E4M3 block scales
                                 [n, k/16]; one fp32 tensor scale per expert matrix;
                                 w = e2m1(q) * e4m3(s) * tensor_scale */
+  MOE_FMT_MXFP4 = 4          /* E2M1 codes [n, k/2] (low nibble first); E8M0 block scales
+                                [n, k/32] (byte c = 2^(c - 127); 255 is NaN); no tensor scale;
+                                w = e2m1(q) * e8m0(s). The 32-element scale block of native
+                                MXFP4 experts (metrale helpers_a.rs, the scale-block note of
+                                transpose_for_prefill_impl) */
 } moe_format;
 
 typedef enum moe_routing {
@@ -86,7 +91,7 @@ typedef enum moe_shared_kind {
 
 /* Layer configuration (plain data; every field is read). */
 typedef struct moe_cfg {
-  int32_t hidden;                /* h: multiple of 8 (of 64 for Q4 and 32 for NVFP4 weights) */
+  int32_t hidden;                /* h: multiple of 8 (of 64 for Q4, 32 for NVFP4 and MXFP4) */
   int32_t num_experts;           /* E */
   int32_t top_k;                 /* k */
   int32_t moe_inter;             /* I: intermediate size of a routed expert */
@@ -107,7 +112,7 @@ typedef struct moe_matrix {
   int32_t format;              /* moe_format */
   int32_t reserved;
   const void* packed;          /* expert 0's weights; 16-byte aligned */
-  const void* scales;          /* Q4: fp16 scales; NVFP4: E4M3 block scales; else NULL */
+  const void* scales;          /* Q4: fp16 scales; NVFP4: E4M3, MXFP4: E8M0 block scales */
   const void* biases;          /* Q4: fp16 biases; else NULL */
   const float* tensor_scale;   /* NVFP4: E floats, one per expert; else NULL */
   int64_t expert_stride;       /* bytes from one expert's weights to the next (multiple of 16) */
@@ -243,6 +248,13 @@ int moe_quantize_q4_affine(const float* w, int n, int k, uint8_t* packed, uint16
  * Outputs: packed [n, k/2], scales [n, k/16] (E4M3 codes), *tensor_scale. */
 int moe_quantize_nvfp4(const float* w, int n, int k, uint8_t* packed, uint8_t* scales,
                        float* tensor_scale);
+
+/* MXFP4 quantisation of one [n, k] matrix, per 32-element block of each row: the shared scale
+ * 2^X with X = floor(log2(max|w_block|)) - 2 (the largest E2M1 magnitude is 6 = 1.5 * 2^2),
+ * clamped to the E8M0 range 2^-127 .. 2^127 (X = 0 for an all-zero block); each element the
+ * nearest E2M1 value of w / 2^X (ties to even, saturating at 6).
+ * Outputs: packed [n, k/2], scales [n, k/32] (E8M0 codes, X + 127). */
+int moe_quantize_mxfp4(const float* w, int n, int k, uint8_t* packed, uint8_t* scales);
 
 /* Decode one [n, k] matrix of `format` from host storage to float32 (test aid). For MOE_FMT_F32
  * and MOE_FMT_BF16 `packed` holds the plain matrix. */

@@ -63,12 +63,13 @@ bool k_ok(int fmt, int k) {
     case MOE_FMT_BF16: return k % 8 == 0;
     case MOE_FMT_Q4_AFFINE_G64: return k % 64 == 0;
     case MOE_FMT_NVFP4: return k % 32 == 0;
+    case MOE_FMT_MXFP4: return k % 32 == 0;
     default: return false;
   }
 }
 
 int check_matrix(const moe_matrix& M, int n, int k, int E, MatDev* out) {
-  if (M.format < MOE_FMT_F32 || M.format > MOE_FMT_NVFP4) return MOE_ERR_BAD_FORMAT;
+  if (M.format < MOE_FMT_F32 || M.format > MOE_FMT_MXFP4) return MOE_ERR_BAD_FORMAT;
   if (!k_ok(M.format, k)) return MOE_ERR_BAD_FORMAT;
   if (!M.packed) return MOE_ERR_NULL_POINTER;
   if (!aligned(M.packed, 16)) return MOE_ERR_MISALIGNED;
@@ -84,9 +85,13 @@ int check_matrix(const moe_matrix& M, int n, int k, int E, MatDev* out) {
     if (!M.scales || !M.tensor_scale) return MOE_ERR_NULL_POINTER;
     if (!aligned(M.scales, 2) || !aligned(M.tensor_scale, 4)) return MOE_ERR_MISALIGNED;
     scale_bytes = (size_t)n * (k / 16);
+  } else if (M.format == MOE_FMT_MXFP4) {
+    if (!M.scales) return MOE_ERR_NULL_POINTER;
+    scale_bytes = (size_t)n * (k / 32);
   }
-  if (scale_bytes && E > 1 && (M.scale_stride < (int64_t)scale_bytes || M.scale_stride % 2))
-    return M.scale_stride % 2 ? MOE_ERR_MISALIGNED : MOE_ERR_BAD_SHAPE;
+  const int64_t salign = M.format == MOE_FMT_MXFP4 ? 1 : 2;  // scale element bytes
+  if (scale_bytes && E > 1 && (M.scale_stride < (int64_t)scale_bytes || M.scale_stride % salign))
+    return M.scale_stride % salign ? MOE_ERR_MISALIGNED : MOE_ERR_BAD_SHAPE;
   out->packed = (const uint8_t*)M.packed;
   out->scales = (const uint8_t*)M.scales;
   out->biases = (const uint8_t*)M.biases;
@@ -191,7 +196,8 @@ cudaError_t launch_gate_up(int fmt, int rb, int grid, size_t smem, cudaStream_t 
     case MOE_FMT_BF16: return launch_gate_up_fmt<MOE_FMT_BF16, XBF16>(rb, grid, smem, st, p);
     case MOE_FMT_Q4_AFFINE_G64:
       return launch_gate_up_fmt<MOE_FMT_Q4_AFFINE_G64, XBF16>(rb, grid, smem, st, p);
-    default: return launch_gate_up_fmt<MOE_FMT_NVFP4, XBF16>(rb, grid, smem, st, p);
+    case MOE_FMT_NVFP4: return launch_gate_up_fmt<MOE_FMT_NVFP4, XBF16>(rb, grid, smem, st, p);
+    default: return launch_gate_up_fmt<MOE_FMT_MXFP4, XBF16>(rb, grid, smem, st, p);
   }
 }
 
@@ -210,7 +216,8 @@ cudaError_t launch_down(int fmt, int rb, int grid, size_t smem, cudaStream_t st,
     case MOE_FMT_F32: return launch_down_fmt<MOE_FMT_F32>(rb, grid, smem, st, p);
     case MOE_FMT_BF16: return launch_down_fmt<MOE_FMT_BF16>(rb, grid, smem, st, p);
     case MOE_FMT_Q4_AFFINE_G64: return launch_down_fmt<MOE_FMT_Q4_AFFINE_G64>(rb, grid, smem, st, p);
-    default: return launch_down_fmt<MOE_FMT_NVFP4>(rb, grid, smem, st, p);
+    case MOE_FMT_NVFP4: return launch_down_fmt<MOE_FMT_NVFP4>(rb, grid, smem, st, p);
+    default: return launch_down_fmt<MOE_FMT_MXFP4>(rb, grid, smem, st, p);
   }
 }
 
@@ -266,7 +273,9 @@ bool plan_fused(const moe_cfg& c, int m, bool has_shared, int fmt, int sms, Fuse
   // scale rows) as the rest of the budget holds, up to every slot a call can have
   const size_t prb = fmt == MOE_FMT_F32 ? (size_t)kmax * 4
                      : fmt == MOE_FMT_BF16 ? (size_t)kmax * 2 : (size_t)kmax / 2;
-  const size_t srb = q4 ? (size_t)(kmax / 64) * 2 : fmt == MOE_FMT_NVFP4 ? (size_t)(kmax / 16) : 0;
+  const size_t srb = q4 ? (size_t)(kmax / 64) * 2
+                     : fmt == MOE_FMT_NVFP4 ? (size_t)(kmax / 16)
+                     : fmt == MOE_FMT_MXFP4 ? (size_t)(kmax / 32) : 0;
   const size_t wblk = align16(cols * prb), sblk = align16(cols * srb);
   const size_t slot_bytes = wblk + (q4 ? 2 * sblk : sblk);
   const int max_slots = (c.top_k * m < c.num_experts ? c.top_k * m : c.num_experts) +
@@ -334,9 +343,9 @@ cudaError_t launch_fused_rb(int m, const Params& p, const FusedPlan& fp, cudaStr
 
 // Formats with a persistent-kernel instantiation (one format for every projection).
 bool fused_formats_ok(int fmt, bool xbf16) {
-  return (fmt == MOE_FMT_F32 && !xbf16) || (xbf16 && (fmt == MOE_FMT_BF16 ||
-                                                      fmt == MOE_FMT_Q4_AFFINE_G64 ||
-                                                      fmt == MOE_FMT_NVFP4));
+  return (fmt == MOE_FMT_F32 && !xbf16) ||
+         (xbf16 && (fmt == MOE_FMT_BF16 || fmt == MOE_FMT_Q4_AFFINE_G64 ||
+                    fmt == MOE_FMT_NVFP4 || fmt == MOE_FMT_MXFP4));
 }
 
 cudaError_t launch_fused(int fmt, bool xbf16, int m, const Params& p, const FusedPlan& fp,
@@ -345,7 +354,8 @@ cudaError_t launch_fused(int fmt, bool xbf16, int m, const Params& p, const Fuse
     case MOE_FMT_F32: return launch_fused_rb<MOE_FMT_F32, false>(m, p, fp, st);
     case MOE_FMT_BF16: return launch_fused_rb<MOE_FMT_BF16, true>(m, p, fp, st);
     case MOE_FMT_Q4_AFFINE_G64: return launch_fused_rb<MOE_FMT_Q4_AFFINE_G64, true>(m, p, fp, st);
-    default: return launch_fused_rb<MOE_FMT_NVFP4, true>(m, p, fp, st);
+    case MOE_FMT_NVFP4: return launch_fused_rb<MOE_FMT_NVFP4, true>(m, p, fp, st);
+    default: return launch_fused_rb<MOE_FMT_MXFP4, true>(m, p, fp, st);
   }
 }
 

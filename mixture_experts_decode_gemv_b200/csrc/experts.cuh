@@ -28,6 +28,7 @@ template <> struct Fmt<MOE_FMT_F32> { static constexpr int kElems = 4; };
 template <> struct Fmt<MOE_FMT_BF16> { static constexpr int kElems = 8; };
 template <> struct Fmt<MOE_FMT_Q4_AFFINE_G64> { static constexpr int kElems = 32; };
 template <> struct Fmt<MOE_FMT_NVFP4> { static constexpr int kElems = 32; };
+template <> struct Fmt<MOE_FMT_MXFP4> { static constexpr int kElems = 32; };
 
 __host__ __device__ constexpr size_t packed_row_bytes(int fmt, int k) {
   return fmt == MOE_FMT_F32 ? (size_t)k * 4 : fmt == MOE_FMT_BF16 ? (size_t)k * 2 : (size_t)k / 2;
@@ -41,6 +42,7 @@ template <> struct Dec<MOE_FMT_F32> { float w[4]; };
 template <> struct Dec<MOE_FMT_BF16> { float w[8]; };
 template <> struct Dec<MOE_FMT_Q4_AFFINE_G64> { float f[32]; float s16, bm; };
 template <> struct Dec<MOE_FMT_NVFP4> { float v[32]; float s0, s1; };
+template <> struct Dec<MOE_FMT_MXFP4> { float v[32]; float s; };
 
 // Row-local pointers of one weight row of one expert matrix.
 struct RowRef {
@@ -63,6 +65,8 @@ __device__ __forceinline__ RowRef row_ref(const MatDev& M, int e, int row) {
   } else if constexpr (FMT == MOE_FMT_NVFP4) {
     r.sc = M.scales + (size_t)e * M.sstride + (size_t)row * (M.k / 16);
     r.ts = __ldg(M.tscale + e);
+  } else if constexpr (FMT == MOE_FMT_MXFP4) {
+    r.sc = M.scales + (size_t)e * M.sstride + (size_t)row * (M.k / 32);
   }
   return r;
 }
@@ -81,6 +85,12 @@ __device__ __forceinline__ uint32_t ldg_u16(const void* p) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t ldg_u8(const void* p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.L2::cache_hint.u8 %0, [%1], %2;" : "=h"(v) : "l"(p), "l"(l2_evict_first()));
+  return v & 0xFFu;
+}
+
 // SMEM: plain loads (the row may live in shared memory or in L2-resident global memory);
 // else streaming non-allocating global loads.
 template <int FMT, bool SMEM>
@@ -95,6 +105,8 @@ __device__ __forceinline__ Chunk load_chunk(const RowRef& rr, int c) {
                << 16);
     } else if constexpr (FMT == MOE_FMT_NVFP4) {
       k.aux = *reinterpret_cast<const unsigned short*>(rr.sc + (size_t)c * 2);
+    } else if constexpr (FMT == MOE_FMT_MXFP4) {
+      k.aux = rr.sc[c];
     }
   } else {
     k.w = ldg_stream(rr.w + (size_t)c * 16);
@@ -102,9 +114,32 @@ __device__ __forceinline__ Chunk load_chunk(const RowRef& rr, int c) {
       k.aux = ldg_u16(rr.sc + (size_t)(c >> 1) * 2) | (ldg_u16(rr.bi + (size_t)(c >> 1) * 2) << 16);
     } else if constexpr (FMT == MOE_FMT_NVFP4) {
       k.aux = ldg_u16(rr.sc + (size_t)c * 2);
+    } else if constexpr (FMT == MOE_FMT_MXFP4) {
+      k.aux = ldg_u8(rr.sc + c);
     }
   }
   return k;
+}
+
+// 32 E2M1 codes of a chunk (byte j: element 2j in the low nibble, 2j+1 in the high nibble) to
+// floats, by the hardware e2m1x2 -> f16x2 conversion.
+__device__ __forceinline__ void decode_e2m1x32(const uint32_t (&q)[4], float (&v)[32]) {
+#pragma unroll
+  for (int t = 0; t < 4; ++t)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const __half2_raw hr = __nv_cvt_fp4x2_to_halfraw2(
+          (__nv_fp4x2_storage_t)((q[t] >> (8 * b)) & 0xFFu), __NV_E2M1);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+      v[8 * t + 2 * b] = f.x;
+      v[8 * t + 2 * b + 1] = f.y;
+    }
+}
+
+// OCP E8M0 scale byte c -> 2^(c - 127) as a float, built from its bits (c = 0 is the subnormal
+// 2^-127; c = 255 is NaN).
+__device__ __forceinline__ float e8m0_to_float(uint32_t c) {
+  return __uint_as_float(c == 0u ? 0x00400000u : c == 0xFFu ? 0x7FC00000u : (c << 23));
 }
 
 template <int FMT>
@@ -129,17 +164,11 @@ __device__ __forceinline__ void decode(const Chunk& ch, Dec<FMT>& d) {
     const float b = __half2float(__ushort_as_half((unsigned short)(ch.aux >> 16)));
     d.s16 = 16.f * s;
     d.bm = b - 16.f * s;
-  } else {  // NVFP4: byte j holds elements 2j (low nibble) and 2j+1 (high nibble)
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const __half2_raw hr = __nv_cvt_fp4x2_to_halfraw2(
-            (__nv_fp4x2_storage_t)((q[t] >> (8 * b)) & 0xFFu), __NV_E2M1);
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-        d.v[8 * t + 2 * b] = f.x;
-        d.v[8 * t + 2 * b + 1] = f.y;
-      }
+  } else if constexpr (FMT == MOE_FMT_MXFP4) {
+    decode_e2m1x32(q, d.v);
+    d.s = e8m0_to_float(ch.aux & 0xFFu);
+  } else {  // NVFP4
+    decode_e2m1x32(q, d.v);
     const __half2_raw hs =
         __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(ch.aux & 0xFFFFu), __NV_E4M3);
     const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&hs));
@@ -155,7 +184,7 @@ __device__ __forceinline__ void decode(const Chunk& ch, Dec<FMT>& d) {
 // quarter-warp's reads hit 8 different bank groups. The arithmetic order is unchanged.
 template <int FMT>
 __device__ __forceinline__ int x_quad(int q) {  // logical quad -> stored quad
-  if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64 || FMT == MOE_FMT_NVFP4) {
+  if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64 || FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_MXFP4) {
     return (q & ~7) | ((q ^ (q >> 3)) & 7);                // 8 quads per chunk
   } else if constexpr (FMT == MOE_FMT_BF16) {
     return (q & ~1) | ((q ^ (q >> 3)) & 1);                // 2 quads per chunk
@@ -214,7 +243,11 @@ __device__ __forceinline__ float dot(const Dec<FMT>& d, const float* row, int c,
       a1 = fmaf(d.v[4 * i + 2], x.z, a1);
       a1 = fmaf(d.v[4 * i + 3], x.w, a1);
     }
-    return fmaf(d.s0, a0, d.s1 * a1);
+    if constexpr (FMT == MOE_FMT_MXFP4) {
+      return (a0 + a1) * d.s;  // one scale for the chunk's 32 elements
+    } else {
+      return fmaf(d.s0, a0, d.s1 * a1);  // NVFP4: one scale per 16
+    }
   }
 }
 

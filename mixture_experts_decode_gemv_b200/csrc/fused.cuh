@@ -280,6 +280,8 @@ __device__ __forceinline__ RowRef tile_row_ref(const MatDev& D, int e, const uin
     r.bi = slot + fp.tile_bi_off + (size_t)lc * (K / 64) * 2;
   } else if constexpr (FMT == MOE_FMT_NVFP4) {
     r.sc = slot + fp.tile_sc_off + (size_t)lc * (K / 16);  // ts: the caller's (staged per slot)
+  } else if constexpr (FMT == MOE_FMT_MXFP4) {
+    r.sc = slot + fp.tile_sc_off + (size_t)lc * (K / 32);
   }
   return r;
 }
@@ -431,6 +433,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
       const size_t prb = packed_row_bytes(FMT, K);
       const size_t srb = FMT == MOE_FMT_Q4_AFFINE_G64 ? (size_t)(K / 64) * 2
                          : FMT == MOE_FMT_NVFP4        ? (size_t)(K / 16)
+                         : FMT == MOE_FMT_MXFP4        ? (size_t)(K / 32)
                                                        : 0;
       const uint8_t* wsrc = D.packed + (size_t)e * D.estride + (size_t)c0 * prb;
       const uint8_t* ssrc = srb ? D.scales + (size_t)e * D.sstride + (size_t)c0 * srb : nullptr;

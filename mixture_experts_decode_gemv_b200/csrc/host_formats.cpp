@@ -2,7 +2,8 @@
 //
 // Minifloat encoders are written from the format definitions: IEEE binary16 (5 exponent bits,
 // bias 15, with infinities), OCP FP8 E4M3 (4 exponent bits, bias 7, no infinity, max 448) and OCP
-// FP4 E2M1 (2 exponent bits, bias 1, max 6). All round to nearest, ties to even.
+// FP4 E2M1 (2 exponent bits, bias 1, max 6). All round to nearest, ties to even. MXFP4 block
+// scales are OCP E8M0 (a biased power of two).
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -91,6 +92,9 @@ static double e2m1_to_double(uint8_t c) {
   return (c & 0x8u) ? -v : v;
 }
 
+// OCP E8M0: an unsigned biased exponent, value 2^(c - 127); 255 encodes NaN.
+static double e8m0_to_double(uint8_t c) { return c == 0xFF ? NAN : std::ldexp(1.0, (int)c - 127); }
+
 static uint16_t f32_to_bf16(float x) {
   uint32_t u;
   std::memcpy(&u, &x, 4);
@@ -124,6 +128,9 @@ extern "C" int moe_packed_bytes(int format, int n, int k, size_t* packed, size_t
     case MOE_FMT_NVFP4:
       if (k % 32) return MOE_ERR_BAD_SHAPE;
       *packed = nk / 2; *scales = nk / 16; *biases = 0; return MOE_OK;
+    case MOE_FMT_MXFP4:
+      if (k % 32) return MOE_ERR_BAD_SHAPE;
+      *packed = nk / 2; *scales = nk / 32; *biases = 0; return MOE_OK;
     default: return MOE_ERR_BAD_FORMAT;
   }
 }
@@ -200,6 +207,31 @@ extern "C" int moe_quantize_nvfp4(const float* w, int n, int k, uint8_t* packed,
   return MOE_OK;
 }
 
+extern "C" int moe_quantize_mxfp4(const float* w, int n, int k, uint8_t* packed,
+                                  uint8_t* scales) {
+  if (!w || !packed || !scales) return MOE_ERR_NULL_POINTER;
+  if (n <= 0 || k <= 0 || k % 32) return MOE_ERR_BAD_SHAPE;
+  const int blocks = k / 32;
+  for (int r = 0; r < n; ++r) {
+    const float* row = w + (size_t)r * k;
+    uint8_t* prow = packed + (size_t)r * (k / 2);
+    for (int b = 0; b < blocks; ++b) {
+      const float* blk = row + b * 32;
+      double bmax = 0.0;
+      for (int j = 0; j < 32; ++j) bmax = std::max(bmax, std::fabs((double)blk[j]));
+      int x = bmax > 0.0 ? (int)std::floor(std::log2(bmax)) - 2 : 0;
+      x = std::min(127, std::max(-127, x));
+      scales[(size_t)r * blocks + b] = (uint8_t)(x + 127);
+      for (int j = 0; j < 32; j += 2) {
+        uint8_t c2[2];
+        for (int t = 0; t < 2; ++t) c2[t] = f64_to_e2m1(std::ldexp((double)blk[j + t], -x));
+        prow[(b * 32 + j) / 2] = (uint8_t)(c2[0] | (c2[1] << 4));
+      }
+    }
+  }
+  return MOE_OK;
+}
+
 extern "C" int moe_dequantize(int format, const void* packed, const void* scales,
                               const void* biases, const float* tensor_scale, int n, int k,
                               float* out) {
@@ -242,6 +274,20 @@ extern "C" int moe_dequantize(int format, const void* packed, const void* scales
           const uint8_t c = (j & 1) ? (byte >> 4) : (byte & 0xF);
           const double sc = e4m3_to_double(s[(size_t)r * (k / 16) + j / 16]);
           out[(size_t)r * k + j] = (float)(e2m1_to_double(c) * sc * ts);
+        }
+      return MOE_OK;
+    }
+    case MOE_FMT_MXFP4: {
+      if (!scales) return MOE_ERR_NULL_POINTER;
+      if (k % 32) return MOE_ERR_BAD_SHAPE;
+      const uint8_t* p = (const uint8_t*)packed;
+      const uint8_t* s = (const uint8_t*)scales;
+      for (int r = 0; r < n; ++r)
+        for (int j = 0; j < k; ++j) {
+          const uint8_t byte = p[(size_t)r * (k / 2) + j / 2];
+          const uint8_t c = (j & 1) ? (byte >> 4) : (byte & 0xF);
+          const double sc = e8m0_to_double(s[(size_t)r * (k / 32) + j / 32]);
+          out[(size_t)r * k + j] = (float)(e2m1_to_double(c) * sc);
         }
       return MOE_OK;
     }

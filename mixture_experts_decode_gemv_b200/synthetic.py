@@ -39,14 +39,17 @@ TAG_SHARED_GATE = 6
 
 PROJ = {"gate": 0, "up": 1, "down": 2}
 
-FORMATS = ("f32", "bf16", "q4_affine_g64", "nvfp4")
+FORMATS = ("f32", "bf16", "q4_affine_g64", "nvfp4", "mxfp4")
 
 # Statistics used to give random codes an N(0, 1/fan_in)-like spread.
 #  - 4-bit affine: codes uniform on 0..15 have variance 255/12 = 21.25 and mean 7.5.
 #  - NVFP4: uniform E2M1 codes have mean-square magnitude 8.5625; block scale codes are drawn
 #    from E4M3 0x30..0x40 (0.5 .. 2.0), mean-square about 1.5, so 0.28 / sqrt(fan_in) as the
 #    per-matrix fp32 scale gives roughly unit-variance logits downstream.
+#  - MXFP4: the same codes; the E8M0 block scale is the power of two nearest to
+#    1 / (sqrt(8.5625 * fan_in)), times 2^-1, 2^0 or 2^1 drawn uniformly per block.
 _Q4_CODE_VAR = 21.25
+_E2M1_MEAN_SQUARE = 8.5625
 _NVFP4_TENSOR_SCALE = 0.28
 _E4M3_SCALE_CODE_LO = 0x30
 _E4M3_SCALE_CODE_HI = 0x40
@@ -108,8 +111,14 @@ LLAMA4_SCOUT = LayerConfig(
     select_on_raw_logits=True, norm_topk_prob=False, weight_before_ffn=True,
     m_list=(1, 16, 64), index=4)
 
+# MXFP4 experts (E2M1 codes with an E8M0 scale per 32 elements) on the Qwen3-30B-A3B shape: the
+# native MXFP4 expert format the pages' prefill helpers handle, at decode sizes.
+QWEN3_30B_A3B_MXFP4 = QWEN3_30B_A3B.replace(name="qwen3_30b_a3b_mxfp4", fmt="mxfp4",
+                                           m_list=(1, 4), index=5)
+
 CONFIGS: Dict[str, LayerConfig] = {
-    c.name: c for c in (TINY, QWEN3_30B_A3B, LFM2_8B_A1B, QWEN3_6_35B_A3B, LLAMA4_SCOUT)
+    c.name: c for c in (TINY, QWEN3_30B_A3B, LFM2_8B_A1B, QWEN3_6_35B_A3B, LLAMA4_SCOUT,
+                        QWEN3_30B_A3B_MXFP4)
 }
 
 
@@ -195,6 +204,13 @@ def draw_matrix(g: np.random.Generator, fmt: str, n: int, k: int, fan_in: int) -
                         dtype=np.uint8)
         ts = np.array([_NVFP4_TENSOR_SCALE / np.sqrt(fan_in)], dtype=np.float32)
         return MatrixSlab(fmt, n, k, _pack_nibbles(codes), scales=sc, tensor_scale=ts)
+    if fmt == "mxfp4":
+        if k % 32:
+            raise ValueError("mxfp4 needs k % 32 == 0")
+        codes = g.integers(0, 16, size=(1, n, k), dtype=np.uint8)
+        base = 127 + int(np.round(-0.5 * np.log2(_E2M1_MEAN_SQUARE * fan_in)))
+        sc = (base + g.integers(-1, 2, size=(1, n, k // 32))).astype(np.uint8)
+        return MatrixSlab(fmt, n, k, _pack_nibbles(codes), scales=sc)
     raise ValueError(f"unknown format {fmt!r}")
 
 
@@ -218,6 +234,9 @@ def _zeros_like_expert(fmt: str, n: int, k: int) -> MatrixSlab:
         return MatrixSlab(fmt, n, k, np.zeros((1, n, k // 2), np.uint8),
                           scales=np.zeros((1, n, k // 16), np.uint8),
                           tensor_scale=np.zeros((1,), np.float32))
+    if fmt == "mxfp4":
+        return MatrixSlab(fmt, n, k, np.zeros((1, n, k // 2), np.uint8),
+                          scales=np.zeros((1, n, k // 32), np.uint8))
     raise ValueError(fmt)
 
 
@@ -341,4 +360,6 @@ def weight_bytes_per_expert(cfg: LayerConfig, inter: Optional[int] = None) -> in
         return n_el // 2 + 4 * (n_el // 64)
     if cfg.fmt == "nvfp4":
         return n_el // 2 + n_el // 16 + 3 * 4
+    if cfg.fmt == "mxfp4":
+        return n_el // 2 + n_el // 32
     raise ValueError(cfg.fmt)

@@ -217,6 +217,35 @@ def test_nvfp4_quantiser_round_trip_bound():
     np.testing.assert_allclose(lib_dec, dec.astype(np.float32), rtol=1e-7, atol=0)
 
 
+def test_mxfp4_quantiser_round_trip_bound():
+    rng = np.random.default_rng(4)
+    n, k = 16, 256
+    w = (rng.standard_normal((n, k)) * 0.05).astype(np.float32)
+    w[3, :32] = 0.0                                   # an all-zero block
+    packed, scales = B.moe_quantize_mxfp4(w)
+    from mixture_experts_decode_gemv_b200.synthetic import MatrixSlab
+    slab = MatrixSlab("mxfp4", n, k, packed[None], scales=scales[None])
+    dec = ref.decode_matrix(slab, 0)
+    # the block scale is 2^(floor(log2 max|w|) - 2): the block maximum lands in [4, 8) on the
+    # E2M1 grid, whose largest value is 6
+    blk = np.repeat(ref.e8m0_value(scales), 32, axis=1)
+    amax = np.abs(w.astype(np.float64)).reshape(n, k // 32, 32).max(axis=2)
+    nz = amax > 0
+    np.testing.assert_array_equal(
+        scales[nz].astype(int) - 127, np.floor(np.log2(amax[nz])).astype(int) - 2)
+    assert scales[3, 0] == 127
+    v = w.astype(np.float64) / blk
+    q = dec / blk
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6])
+    step = np.where(np.abs(v) < 2, 0.25, np.where(np.abs(v) < 4, 0.5, 1.0))
+    err = np.abs(q - v)
+    assert np.all(err <= step + np.maximum(0, np.abs(v) - 6) + 1e-9)
+    assert np.all(np.isin(np.abs(q), grid))
+    lib_dec = B.moe_dequantize(B.MOE_FMT_MXFP4, packed, scales, None, None, n, k)
+    np.testing.assert_array_equal(lib_dec, dec.astype(np.float32))
+    assert B.moe_packed_bytes(B.MOE_FMT_MXFP4, 10, 128) == (640, 40, 0)
+
+
 def test_dequantize_bf16_and_f32_plain():
     w = np.arange(12, dtype=np.float32).reshape(3, 4) - 5.5
     np.testing.assert_array_equal(B.moe_dequantize(B.MOE_FMT_F32, w, None, None, None, 3, 4), w)

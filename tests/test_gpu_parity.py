@@ -41,6 +41,10 @@ SMALL = {
                                   select_on_raw_logits=True, norm_topk_prob=True, index=206),
     "max_experts": LayerConfig(name="max_experts", hidden=64, num_experts=256, top_k=8,
                                moe_inter=32, fmt="bf16", index=207),
+    "ragged_mxfp4": LayerConfig(name="ragged_mxfp4", hidden=160, num_experts=6, top_k=2,
+                                moe_inter=96, shared_inter=64, shared_kind="plain", fmt="mxfp4",
+                                routing="sigmoid", has_expert_bias=True,
+                                routed_scaling_factor=1.5, index=208),
 }
 
 _CACHE = {}
@@ -220,7 +224,8 @@ class _Path:
             os.environ["MOE_DECODE_PATH"] = self.old
 
 
-PATH_CASES = [(n, m) for n in ("qwen3_30b_a3b", "lfm2_8b_a1b", "qwen3_6_35b_a3b", "llama4_scout")
+PATH_CASES = [(n, m) for n in ("qwen3_30b_a3b", "lfm2_8b_a1b", "qwen3_6_35b_a3b", "llama4_scout",
+                                "qwen3_30b_a3b_mxfp4")
               for m in (1, 2, 3, 4)] + [(n, m) for n in SMALL for m in (1, 4)]
 
 
