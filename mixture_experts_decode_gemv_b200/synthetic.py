@@ -39,7 +39,7 @@ TAG_SHARED_GATE = 6
 
 PROJ = {"gate": 0, "up": 1, "down": 2}
 
-FORMATS = ("f32", "bf16", "q4_affine_g64", "nvfp4", "mxfp4")
+FORMATS = ("f32", "bf16", "q4_affine_g64", "nvfp4", "mxfp4", "fp8_e4m3")
 
 # Statistics used to give random codes an N(0, 1/fan_in)-like spread.
 #  - 4-bit affine: codes uniform on 0..15 have variance 255/12 = 21.25 and mean 7.5.
@@ -48,8 +48,12 @@ FORMATS = ("f32", "bf16", "q4_affine_g64", "nvfp4", "mxfp4")
 #    per-matrix fp32 scale gives roughly unit-variance logits downstream.
 #  - MXFP4: the same codes; the E8M0 block scale is the power of two nearest to
 #    1 / (sqrt(8.5625 * fan_in)), times 2^-1, 2^0 or 2^1 drawn uniformly per block.
+#  - FP8 E4M3: random sign, exponent field uniform on 5..9 (2^-2 .. 2^2) and mantissa uniform on
+#    0..7 (no NaN codes); mean-square value 4.2625 * 2.1484375, so the per-matrix fp32 scale
+#    1 / sqrt(that * fan_in) gives variance 1 / fan_in.
 _Q4_CODE_VAR = 21.25
 _E2M1_MEAN_SQUARE = 8.5625
+_E4M3_DRAWN_MEAN_SQUARE = ((1 / 16 + 1 / 4 + 1 + 4 + 16) / 5) * (1100 / 8 / 64)
 _NVFP4_TENSOR_SCALE = 0.28
 _E4M3_SCALE_CODE_LO = 0x30
 _E4M3_SCALE_CODE_HI = 0x40
@@ -67,13 +71,14 @@ class LayerConfig:
     shared_inter: int = 0
     fmt: str = "bf16"              # routed and shared expert weight format
     x_dtype: str = "bf16"          # activations, router matrix and shared gate vector
-    routing: str = "softmax"       # "softmax" | "sigmoid"
+    routing: str = "softmax"       # "softmax" | "sigmoid" | "sqrtsoftplus"
     norm_topk_prob: bool = True
     select_on_raw_logits: bool = False
     has_expert_bias: bool = False
     routed_scaling_factor: float = 1.0
     weight_before_ffn: bool = False
     shared_kind: str = "none"      # "none" | "plain" | "sigmoid_gate"
+    activation: str = "swiglu"     # "swiglu" (silu(g) * u) | "geglu" (gelu_tanh(g) * u)
     m_list: Tuple[int, ...] = (1,)
     index: int = 0                 # seed = SEED_BASE + index
 
@@ -154,8 +159,8 @@ def _pack_nibbles(codes: np.ndarray) -> np.ndarray:
 class MatrixSlab:
     """One projection of E experts, each an ``[n, k]`` matrix, in the library's storage.
 
-    ``data``: f32 -> float32 ``[E, n, k]``; bf16 -> uint16 ``[E, n, k]``; 4-bit formats -> uint8
-    ``[E, n, k/2]``. ``scales``: q4 -> fp16 bits ``[E, n, k/64]``; nvfp4 -> E4M3 codes
+    ``data``: f32 -> float32 ``[E, n, k]``; bf16 -> uint16 ``[E, n, k]``; fp8_e4m3 -> uint8
+    ``[E, n, k]``; 4-bit formats -> uint8 ``[E, n, k/2]``. ``scales``: q4 -> fp16 bits ``[E, n, k/64]``; nvfp4 -> E4M3 codes
     ``[E, n, k/16]``. ``biases``: q4 -> fp16 bits ``[E, n, k/64]``. ``tensor_scale``: nvfp4 ->
     float32 ``[E]``.
     """
@@ -204,6 +209,15 @@ def draw_matrix(g: np.random.Generator, fmt: str, n: int, k: int, fan_in: int) -
                         dtype=np.uint8)
         ts = np.array([_NVFP4_TENSOR_SCALE / np.sqrt(fan_in)], dtype=np.float32)
         return MatrixSlab(fmt, n, k, _pack_nibbles(codes), scales=sc, tensor_scale=ts)
+    if fmt == "fp8_e4m3":
+        if k % 16:
+            raise ValueError("fp8_e4m3 needs k % 16 == 0")
+        sign = g.integers(0, 2, size=(1, n, k), dtype=np.uint8)
+        expo = g.integers(5, 10, size=(1, n, k), dtype=np.uint8)
+        mant = g.integers(0, 8, size=(1, n, k), dtype=np.uint8)
+        codes = ((sign << np.uint8(7)) | (expo << np.uint8(3)) | mant).astype(np.uint8)
+        ts = np.array([1.0 / np.sqrt(_E4M3_DRAWN_MEAN_SQUARE * fan_in)], dtype=np.float32)
+        return MatrixSlab(fmt, n, k, codes, tensor_scale=ts)
     if fmt == "mxfp4":
         if k % 32:
             raise ValueError("mxfp4 needs k % 32 == 0")
@@ -237,6 +251,9 @@ def _zeros_like_expert(fmt: str, n: int, k: int) -> MatrixSlab:
     if fmt == "mxfp4":
         return MatrixSlab(fmt, n, k, np.zeros((1, n, k // 2), np.uint8),
                           scales=np.zeros((1, n, k // 32), np.uint8))
+    if fmt == "fp8_e4m3":
+        return MatrixSlab(fmt, n, k, np.zeros((1, n, k), np.uint8),
+                          tensor_scale=np.zeros((1,), np.float32))
     raise ValueError(fmt)
 
 
@@ -362,4 +379,6 @@ def weight_bytes_per_expert(cfg: LayerConfig, inter: Optional[int] = None) -> in
         return n_el // 2 + n_el // 16 + 3 * 4
     if cfg.fmt == "mxfp4":
         return n_el // 2 + n_el // 32
+    if cfg.fmt == "fp8_e4m3":
+        return n_el + 3 * 4
     raise ValueError(cfg.fmt)

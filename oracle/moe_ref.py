@@ -19,6 +19,9 @@ What it computes, per row r, with the sources it follows:
      on raw logits (frink-models ``routed_weight_site.rs`` module doc: Llama 4 takes the top-k of
      the raw logits, the same experts as on the sigmoid probabilities), else sigmoid(l).
    The k largest keys win; equal keys go to the lower expert id; slots are in descending key order.
+   The sqrt-softplus router (iron PR, the ``router_sqrtsoftplus`` kernel of the moe family)
+   ranks and weights like the sigmoid router with the score sqrt(softplus(l)) = sqrt(log(1+e^l))
+   in place of sigmoid(l); the page names the router only, this is the plain reading of its name.
 3. Routing weights: softmax probability (over all E) or unbiased sigmoid score of each selected
    expert, divided by their sum when ``norm_topk_prob``, then multiplied by
    ``routed_scaling_factor`` (mlxcel PR "perf(moe): wire lfm2 to the fused decode-MoE kernel":
@@ -26,7 +29,10 @@ What it computes, per row r, with the sources it follows:
 4. Routed-weight site (frink-models ``routed_weight_site.rs``, ``routed_slot``): the slot's
    expert input is x and its output carries w, or, when the weight sits before the FFN (Llama 4),
    the input is w*x and the output carries 1.
-5. Expert: ``down(silu(gate(x~)) * up(x~))`` with silu(z) = z * sigmoid(z).
+5. Expert: ``down(silu(gate(x~)) * up(x~))`` with silu(z) = z * sigmoid(z); with the GeGLU
+   activation (metrale ``helpers_a.rs``, ``set_gelu_activation``: the expert activation becomes
+   ``gelu_mul``) the gate goes through GELU instead, in its tanh form (the form of the Gemma
+   models that page wires it for).
 6. Output: the sum over slots (in slot order) of weight * expert output, plus the shared expert,
    scaled by sigmoid(w_sg . x_r) for a sigmoid-gated shared expert (metrale
    ``forward_bf16_grouped_decode.rs``: the blend receives the layer input and the shared expert
@@ -43,6 +49,9 @@ Weight formats decoded here (storage defined by the library's pack helpers; 4-bi
  * NVFP4: E2M1 codes, one E4M3 scale per 16 elements (the NVFP4 scale block of metrale
    ``helpers_a.rs``), one fp32 tensor scale per matrix (its ``weight_scale_2``):
    ``w = e2m1(q) * e4m3(s) * tensor_scale``;
+ * FP8: E4M3 codes ``[n, k]`` (one byte per element) and one fp32 scale per expert matrix
+   (the FP8 grouped decode of metrale ``forward_fp8_grouped_decode.rs``, whose scale layout
+   the pages do not give; read as one scale per matrix): ``w = e4m3(q) * scale``;
  * MXFP4: E2M1 codes, one E8M0 scale per 32 elements (the native MXFP4 scale block of metrale
    ``helpers_a.rs``, the scale-block note of ``transpose_for_prefill_impl``), no tensor scale:
    ``w = e2m1(q) * 2**(s - 127)`` (E8M0 as the OCP Microscaling specification defines it).
@@ -139,6 +148,9 @@ def decode_matrix(slab, e: int = 0) -> np.ndarray:
     if slab.fmt == "mxfp4":
         v = e2m1_value(unpack_nibbles(slab.data[e], k))
         return v * np.repeat(e8m0_value(slab.scales[e]), 32, axis=1)
+    if slab.fmt == "fp8_e4m3":
+        v = e4m3_value(np.asarray(slab.data[e], dtype=np.uint8).reshape(n, k))
+        return v * float(np.float32(slab.tensor_scale[e]))
     raise ValueError(f"unknown format {slab.fmt!r}")
 
 
@@ -175,6 +187,32 @@ def silu(z):
     return z * sigmoid(z)
 
 
+def softplus(z):
+    """softplus(z) = log(1 + e^z), written as max(z, 0) + log1p(e^-|z|) (no overflow)."""
+    z = np.asarray(z, dtype=np.float64)
+    return np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
+
+
+def sqrtsoftplus(z):
+    """The sqrt-softplus router score: sqrt(softplus(z)) (a positive, increasing score)."""
+    return np.sqrt(softplus(z))
+
+
+def gelu_tanh(z):
+    """GELU in its tanh form: z/2 * (1 + tanh(sqrt(2/pi) * (z + 0.044715 z^3)))."""
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * z * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (z + 0.044715 * z ** 3)))
+
+
+def router_score(l, routing: str):
+    """Per-expert score of the non-softmax routers: sigmoid or sqrt-softplus of the logit."""
+    if routing == "sigmoid":
+        return sigmoid(l)
+    if routing == "sqrtsoftplus":
+        return sqrtsoftplus(l)
+    raise ValueError(routing)
+
+
 def router_logits(x64: np.ndarray, wr64: np.ndarray) -> np.ndarray:
     """``[m, h] x [E, h] -> [m, E]``, one matrix-vector product per row."""
     return np.stack([wr64 @ np.array(row) for row in x64])
@@ -185,11 +223,11 @@ def selection_keys(logits_row: np.ndarray, cfg, expert_bias: Optional[np.ndarray
     l = np.asarray(logits_row, dtype=np.float64)
     if cfg.routing == "softmax":
         return l.copy()
-    if cfg.routing != "sigmoid":
+    if cfg.routing not in ("sigmoid", "sqrtsoftplus"):
         raise ValueError(cfg.routing)
     if cfg.select_on_raw_logits:
         return l.copy()
-    s = sigmoid(l)
+    s = router_score(l, cfg.routing)
     if cfg.has_expert_bias:
         return s + np.asarray(expert_bias, dtype=np.float32).astype(np.float64)
     return s
@@ -209,7 +247,7 @@ def routing_weights(logits_row: np.ndarray, ids: Sequence[int], cfg) -> np.ndarr
         p /= p.sum()
         w = p[list(ids)]
     else:
-        w = sigmoid(l[list(ids)])
+        w = router_score(l[list(ids)], cfg.routing)
     if cfg.norm_topk_prob:
         w = w / w.sum()
     return w * float(np.float32(cfg.routed_scaling_factor))
@@ -261,11 +299,19 @@ def group_by_expert(idx: np.ndarray, num_experts: int) -> Dict[str, np.ndarray]:
 # ---------------------------------------------------------------------------------------------
 
 
-def swiglu_expert(wg: np.ndarray, wu: np.ndarray, wd: np.ndarray, xin: np.ndarray) -> np.ndarray:
-    """``down(silu(gate(x)) * up(x))`` for one input vector."""
+def swiglu_expert(wg: np.ndarray, wu: np.ndarray, wd: np.ndarray, xin: np.ndarray,
+                  activation: str = "swiglu") -> np.ndarray:
+    """``down(silu(gate(x)) * up(x))`` for one input vector; with ``activation="geglu"`` the gate
+    goes through GELU (tanh form) instead of SiLU."""
     xin = np.array(xin, dtype=np.float64)
-    act = silu(wg @ xin) * (wu @ xin)
-    return wd @ act
+    g = wg @ xin
+    if activation == "swiglu":
+        a = silu(g)
+    elif activation == "geglu":
+        a = gelu_tanh(g)
+    else:
+        raise ValueError(activation)
+    return wd @ (a * (wu @ xin))
 
 
 class OracleLayer:
@@ -358,7 +404,7 @@ def moe_forward(layer: OracleLayer, x: np.ndarray, rows: Optional[Sequence[int]]
         wg, wu, wd = layer.expert(e)
         for r, s in users[e]:
             xin, omega = routed_slot(x64[r], w[r, s], cfg.weight_before_ffn)
-            y[(r, s)] = swiglu_expert(wg, wu, wd, xin)
+            y[(r, s)] = swiglu_expert(wg, wu, wd, xin, cfg.activation)
             weight_site[(r, s)] = omega
     out = np.zeros((len(rows), cfg.hidden), dtype=np.float64)
     for i, r in enumerate(rows):
@@ -370,7 +416,7 @@ def moe_forward(layer: OracleLayer, x: np.ndarray, rows: Optional[Sequence[int]]
         sg, su, sd = layer.shared()
         for i, r in enumerate(rows):
             g = 1.0 if gamma is None else gamma[r]
-            out[i] = out[i] + g * swiglu_expert(sg, su, sd, x64[r])
+            out[i] = out[i] + g * swiglu_expert(sg, su, sd, x64[r], cfg.activation)
     aux = dict(rt)
     aux.update(group_by_expert(idx, cfg.num_experts))
     return out, aux

@@ -157,3 +157,17 @@ def test_mxfp4_with_unit_scales_is_plain_e2m1_and_scales_by_powers_of_two():
                                          scales=np.full_like(sc, 0x7F)), 0)
     np.testing.assert_array_equal(plain, ref.e2m1_value(q))
     np.testing.assert_array_equal(w, plain * np.exp2(np.repeat(sc[0].astype(float) - 127, 32, 1)))
+
+
+def test_fp8_e4m3_hand_built(golden_dir):
+    codes, vals = _read_table(os.path.join(golden_dir, "e4m3_values.txt"))
+    ok = ~np.isnan(vals)
+    row = codes[ok].astype(np.uint8)
+    k = 16
+    data = np.zeros((1, 2, k), np.uint8)
+    data[0, 0, :row.size] = row
+    data[0, 1, :] = 0x38                                       # 1.0 everywhere
+    slab = MatrixSlab("fp8_e4m3", 2, k, data, tensor_scale=np.array([0.5], np.float32))
+    w = ref.decode_matrix(slab, 0)
+    np.testing.assert_array_equal(w[0, :row.size], vals[ok] * 0.5)
+    np.testing.assert_array_equal(w[1], 0.5)

@@ -190,3 +190,21 @@ def test_published_shapes_meet_the_gap_rule(name):
     for r in range(POOL_ROWS):
         keys = np.sort(key_fn(x[r]))[::-1][: min(k + 1, cfg.num_experts)]
         assert np.min(keys[:-1] - keys[1:]) >= GAP_MIN
+
+
+def test_gelu_tanh_matches_the_library_and_closed_forms():
+    import torch
+    assert ref.gelu_tanh(0.0) == 0.0
+    z = np.linspace(-12, 12, 2401)
+    lib = torch.nn.functional.gelu(torch.tensor(z, dtype=torch.float64), approximate="tanh")
+    np.testing.assert_allclose(ref.gelu_tanh(z), lib.numpy(), rtol=1e-13, atol=1e-15)
+    # odd part: gelu(z) - gelu(-z) = z
+    np.testing.assert_allclose(ref.gelu_tanh(z) - ref.gelu_tanh(-z), z, rtol=0, atol=1e-12)
+
+
+def test_geglu_expert_with_identity_matrices():
+    x = np.array([0.0, 1.0, -2.0, 3.5])
+    eye = np.eye(4)
+    y = ref.swiglu_expert(eye, eye, eye, x, "geglu")
+    np.testing.assert_allclose(y, ref.gelu_tanh(x) * x, rtol=1e-15)
+    assert not np.allclose(y, ref.swiglu_expert(eye, eye, eye, x))

@@ -179,3 +179,43 @@ def test_grouping_matches_counting_sort():
         active = [e for e in range(E) if offsets[e + 1] > offsets[e]]
         assert list(g["active"]) == active
         assert g["active_count"] == len(active) <= min(te, E)
+
+
+# ---- sqrt-softplus router ----------------------------------------------------------------------
+
+def test_sqrtsoftplus_closed_forms_and_library_softplus():
+    import torch
+    # softplus(0) = ln 2, so the score at 0 is sqrt(ln 2)
+    assert ref.sqrtsoftplus(0.0) == math.sqrt(math.log(2.0))
+    z = np.linspace(-40, 40, 801)
+    # torch switches to the identity above `threshold` (default 20): move it out of the way
+    lib = torch.nn.functional.softplus(torch.tensor(z, dtype=torch.float64), threshold=1e4).numpy()
+    np.testing.assert_allclose(ref.softplus(z), lib, rtol=1e-14, atol=1e-300)
+    # softplus(z) - softplus(-z) = z; large z: score -> sqrt(z); very negative z: score -> e^(z/2)
+    np.testing.assert_allclose(ref.softplus(z) - ref.softplus(-z), z, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(ref.sqrtsoftplus(60.0), math.sqrt(60.0), rtol=1e-15)
+    np.testing.assert_allclose(ref.sqrtsoftplus(-60.0), math.exp(-30.0), rtol=1e-12)
+
+
+def test_sqrtsoftplus_routing_selects_like_raw_logits_and_weights_by_score():
+    rng = np.random.default_rng(11)
+    cfg = cfg_of(num_experts=16, top_k=4, routing="sqrtsoftplus", norm_topk_prob=False)
+    for _ in range(50):
+        l = rng.standard_normal(16) * 3
+        ids, w = ref.route_row(l, cfg, None)
+        assert ids == list(np.argsort(-l, kind="stable")[:4])     # an increasing score
+        np.testing.assert_allclose(w, np.sqrt(np.log1p(np.exp(l[ids]))), rtol=1e-14)
+    cfg_n = cfg_of(num_experts=16, top_k=4, routing="sqrtsoftplus", norm_topk_prob=True,
+                   routed_scaling_factor=2.0)
+    ids, w = ref.route_row(l, cfg_n, None)
+    np.testing.assert_allclose(w.sum(), 2.0, rtol=1e-14)
+
+
+def test_sqrtsoftplus_bias_changes_the_set_not_the_weights():
+    cfg = cfg_of(num_experts=4, top_k=1, routing="sqrtsoftplus", has_expert_bias=True,
+                 norm_topk_prob=False)
+    l = np.array([0.5, 0.4, -1.0, 0.0])
+    bias = np.array([0.0, 0.5, 0.0, 0.0], dtype=np.float32)
+    ids, w = ref.route_row(l, cfg, bias)
+    assert ids == [1]                                           # 0.4 + bias beats 0.5
+    np.testing.assert_allclose(w, [math.sqrt(math.log1p(math.exp(0.4)))], rtol=1e-15)
