@@ -70,18 +70,32 @@ typedef enum moe_format {
   MOE_FMT_NVFP4 = 3,         /* E2M1 codes [n, k/2] (low nibble first); E4M3 block scales
                                 [n, k/16]; one fp32 tensor scale per expert matrix;
                                 w = e2m1(q) * e4m3(s) * tensor_scale */
-  MOE_FMT_MXFP4 = 4          /* E2M1 codes [n, k/2] (low nibble first); E8M0 block scales
+  MOE_FMT_MXFP4 = 4,         /* E2M1 codes [n, k/2] (low nibble first); E8M0 block scales
                                 [n, k/32] (byte c = 2^(c - 127); 255 is NaN); no tensor scale;
                                 w = e2m1(q) * e8m0(s). The 32-element scale block of native
                                 MXFP4 experts (metrale helpers_a.rs, the scale-block note of
                                 transpose_for_prefill_impl) */
+  MOE_FMT_FP8_E4M3 = 5       /* OCP E4M3 codes [n, k], one byte per element; one fp32 scale per
+                                expert matrix in tensor_scale; w = e4m3(q) * tensor_scale (the
+                                FP8 grouped decode of metrale forward_fp8_grouped_decode.rs;
+                                the pages give no scale layout, read as per matrix) */
 } moe_format;
 
 typedef enum moe_routing {
   MOE_ROUTE_SOFTMAX = 0, /* p = softmax(l) over all experts, select by l, weight p */
-  MOE_ROUTE_SIGMOID = 1  /* s = sigmoid(l); select by s + expert_bias (if any), by l when
+  MOE_ROUTE_SIGMOID = 1, /* s = sigmoid(l); select by s + expert_bias (if any), by l when
                             select_on_raw_logits, else by s; weight s (never the bias) */
+  MOE_ROUTE_SQRTSOFTPLUS = 2 /* as MOE_ROUTE_SIGMOID with s = sqrt(softplus(l))
+                                = sqrt(log(1 + e^l)) (the router_sqrtsoftplus kernel named by
+                                the iron PR; its formula is the plain reading of the name) */
 } moe_routing;
+
+typedef enum moe_activation {
+  MOE_ACT_SWIGLU = 0,  /* act = silu(g) * u, silu(z) = z * sigmoid(z) */
+  MOE_ACT_GEGLU = 1    /* act = gelu(g) * u with GELU in its tanh form,
+                          z/2 * (1 + tanh(sqrt(2/pi) * (z + 0.044715 z^3))) (metrale helpers_a.rs,
+                          set_gelu_activation: the expert activation becomes gelu_mul) */
+} moe_activation;
 
 typedef enum moe_shared_kind {
   MOE_SHARED_NONE = 0,
@@ -98,13 +112,14 @@ typedef struct moe_cfg {
   int32_t shared_inter;          /* S: intermediate size of the shared expert (0 = none) */
   int32_t routing;               /* moe_routing */
   int32_t norm_topk_prob;        /* 1: divide the k weights by their sum */
-  int32_t select_on_raw_logits;  /* 1 (sigmoid only): rank by the raw logit */
-  int32_t has_expert_bias;       /* 1 (sigmoid only): rank by sigmoid(l) + expert_bias[e] */
+  int32_t select_on_raw_logits;  /* 1 (sigmoid, sqrt-softplus): rank by the raw logit */
+  int32_t has_expert_bias;       /* 1 (sigmoid, sqrt-softplus): rank by score(l) + bias[e] */
   float routed_scaling_factor;   /* multiplies every routing weight (after normalisation) */
   int32_t weight_before_ffn;     /* 1: the weight scales the expert input, the output carries 1 */
   int32_t shared_kind;           /* moe_shared_kind */
   int32_t x_dtype;               /* MOE_FMT_F32 or MOE_FMT_BF16: x, router_w and shared gate */
   int32_t out_dtype;             /* MOE_FMT_F32 or MOE_FMT_BF16 (round to nearest even) */
+  int32_t activation;            /* moe_activation of the routed and shared experts */
 } moe_cfg;
 
 /* One projection of all experts (or of the shared expert, E = 1). Device pointers. */
@@ -114,7 +129,7 @@ typedef struct moe_matrix {
   const void* packed;          /* expert 0's weights; 16-byte aligned */
   const void* scales;          /* Q4: fp16 scales; NVFP4: E4M3, MXFP4: E8M0 block scales */
   const void* biases;          /* Q4: fp16 biases; else NULL */
-  const float* tensor_scale;   /* NVFP4: E floats, one per expert; else NULL */
+  const float* tensor_scale;   /* NVFP4 and FP8: E floats, one per expert; else NULL */
   int64_t expert_stride;       /* bytes from one expert's weights to the next (multiple of 16) */
   int64_t scale_stride;        /* bytes from one expert's scales (and biases) to the next */
 } moe_matrix;
@@ -255,6 +270,11 @@ int moe_quantize_nvfp4(const float* w, int n, int k, uint8_t* packed, uint8_t* s
  * nearest E2M1 value of w / 2^X (ties to even, saturating at 6).
  * Outputs: packed [n, k/2], scales [n, k/32] (E8M0 codes, X + 127). */
 int moe_quantize_mxfp4(const float* w, int n, int k, uint8_t* packed, uint8_t* scales);
+
+/* FP8 E4M3 quantisation of one [n, k] matrix: tensor_scale = max|w| / 448 (1 for an all-zero
+ * matrix); each element the nearest E4M3 value of w / tensor_scale (ties to even, saturating at
+ * 448). Outputs: packed [n, k] (E4M3 codes), *tensor_scale. */
+int moe_quantize_fp8_e4m3(const float* w, int n, int k, uint8_t* packed, float* tensor_scale);
 
 /* Decode one [n, k] matrix of `format` from host storage to float32 (test aid). For MOE_FMT_F32
  * and MOE_FMT_BF16 `packed` holds the plain matrix. */

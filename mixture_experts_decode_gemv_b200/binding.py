@@ -33,13 +33,17 @@ MOE_MAX_ROWS = 64
 MOE_MAX_EXPERTS = 256
 MOE_MAX_TOP_K = 8
 
-MOE_FMT_F32, MOE_FMT_BF16, MOE_FMT_Q4_AFFINE_G64, MOE_FMT_NVFP4, MOE_FMT_MXFP4 = 0, 1, 2, 3, 4
-MOE_ROUTE_SOFTMAX, MOE_ROUTE_SIGMOID = 0, 1
+(MOE_FMT_F32, MOE_FMT_BF16, MOE_FMT_Q4_AFFINE_G64, MOE_FMT_NVFP4, MOE_FMT_MXFP4,
+ MOE_FMT_FP8_E4M3) = 0, 1, 2, 3, 4, 5
+MOE_ROUTE_SOFTMAX, MOE_ROUTE_SIGMOID, MOE_ROUTE_SQRTSOFTPLUS = 0, 1, 2
+MOE_ACT_SWIGLU, MOE_ACT_GEGLU = 0, 1
 MOE_SHARED_NONE, MOE_SHARED_PLAIN, MOE_SHARED_SIGMOID_GATE = 0, 1, 2
 
 FORMAT_CODES = {"f32": MOE_FMT_F32, "bf16": MOE_FMT_BF16, "q4_affine_g64": MOE_FMT_Q4_AFFINE_G64,
-                "nvfp4": MOE_FMT_NVFP4, "mxfp4": MOE_FMT_MXFP4}
-ROUTING_CODES = {"softmax": MOE_ROUTE_SOFTMAX, "sigmoid": MOE_ROUTE_SIGMOID}
+                "nvfp4": MOE_FMT_NVFP4, "mxfp4": MOE_FMT_MXFP4, "fp8_e4m3": MOE_FMT_FP8_E4M3}
+ROUTING_CODES = {"softmax": MOE_ROUTE_SOFTMAX, "sigmoid": MOE_ROUTE_SIGMOID,
+                 "sqrtsoftplus": MOE_ROUTE_SQRTSOFTPLUS}
+ACTIVATION_CODES = {"swiglu": MOE_ACT_SWIGLU, "geglu": MOE_ACT_GEGLU}
 SHARED_CODES = {"none": MOE_SHARED_NONE, "plain": MOE_SHARED_PLAIN,
                 "sigmoid_gate": MOE_SHARED_SIGMOID_GATE}
 
@@ -49,7 +53,7 @@ EXPORTS = (
     "moe_get_device_status", "moe_packed_bytes", "moe_pack_bf16", "moe_quantize_q4_affine",
     "moe_quantize_nvfp4", "moe_dequantize", "moe_status_string", "moe_last_cuda_error",
     "moe_version", "moe_decode_forward_no_alloc", "moe_decode_launches",
-    "moe_debug_barrier_test", "moe_quantize_mxfp4",
+    "moe_debug_barrier_test", "moe_quantize_mxfp4", "moe_quantize_fp8_e4m3",
 )
 
 MOE_NO_ALLOC_SCRATCH_BYTES = 16 << 20
@@ -72,7 +76,7 @@ class moe_cfg(ctypes.Structure):
         ("select_on_raw_logits", ctypes.c_int32), ("has_expert_bias", ctypes.c_int32),
         ("routed_scaling_factor", ctypes.c_float), ("weight_before_ffn", ctypes.c_int32),
         ("shared_kind", ctypes.c_int32), ("x_dtype", ctypes.c_int32),
-        ("out_dtype", ctypes.c_int32),
+        ("out_dtype", ctypes.c_int32), ("activation", ctypes.c_int32),
     ]
 
 
@@ -109,6 +113,7 @@ def _load() -> ctypes.CDLL:
         "moe_quantize_q4_affine": [vp, i32, i32, vp, vp, vp],
         "moe_quantize_nvfp4": [vp, i32, i32, vp, vp, vp],
         "moe_quantize_mxfp4": [vp, i32, i32, vp, vp],
+        "moe_quantize_fp8_e4m3": [vp, i32, i32, vp, vp],
         "moe_dequantize": [i32, vp, vp, vp, vp, i32, i32, vp],
         "moe_decode_forward_no_alloc": [P(moe_cfg), i32, vp, vp, vp, P(moe_expert_table),
                                         P(moe_expert_table), vp, vp, vp],
@@ -285,6 +290,16 @@ def moe_quantize_mxfp4(w: np.ndarray):
     _check(lib.moe_quantize_mxfp4(w.ctypes.data, n, k, packed.ctypes.data, scales.ctypes.data),
            "moe_quantize_mxfp4")
     return packed, scales
+
+
+def moe_quantize_fp8_e4m3(w: np.ndarray):
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    n, k = w.shape
+    packed = np.empty((n, k), np.uint8)
+    ts = np.zeros(1, np.float32)
+    _check(lib.moe_quantize_fp8_e4m3(w.ctypes.data, n, k, packed.ctypes.data, ts.ctypes.data),
+           "moe_quantize_fp8_e4m3")
+    return packed, ts
 
 
 def moe_dequantize(fmt: int, packed: np.ndarray, scales, biases, tensor_scale, n: int, k: int):

@@ -37,7 +37,8 @@ int check_cfg(const moe_cfg* c, int m) {
   if (c->top_k < 1 || c->top_k > MOE_MAX_TOP_K || c->top_k > c->num_experts)
     return MOE_ERR_BAD_SHAPE;
   if (c->moe_inter <= 0 || c->moe_inter % 4 || c->shared_inter < 0) return MOE_ERR_BAD_SHAPE;
-  if (c->routing != MOE_ROUTE_SOFTMAX && c->routing != MOE_ROUTE_SIGMOID) return MOE_ERR_BAD_OPTION;
+  if (c->routing < MOE_ROUTE_SOFTMAX || c->routing > MOE_ROUTE_SQRTSOFTPLUS) return MOE_ERR_BAD_OPTION;
+  if (c->activation != MOE_ACT_SWIGLU && c->activation != MOE_ACT_GEGLU) return MOE_ERR_BAD_OPTION;
   auto is01 = [](int v) { return v == 0 || v == 1; };
   if (!is01(c->norm_topk_prob) || !is01(c->select_on_raw_logits) || !is01(c->has_expert_bias) ||
       !is01(c->weight_before_ffn))
@@ -64,12 +65,13 @@ bool k_ok(int fmt, int k) {
     case MOE_FMT_Q4_AFFINE_G64: return k % 64 == 0;
     case MOE_FMT_NVFP4: return k % 32 == 0;
     case MOE_FMT_MXFP4: return k % 32 == 0;
+    case MOE_FMT_FP8_E4M3: return k % 16 == 0;
     default: return false;
   }
 }
 
 int check_matrix(const moe_matrix& M, int n, int k, int E, MatDev* out) {
-  if (M.format < MOE_FMT_F32 || M.format > MOE_FMT_MXFP4) return MOE_ERR_BAD_FORMAT;
+  if (M.format < MOE_FMT_F32 || M.format > MOE_FMT_FP8_E4M3) return MOE_ERR_BAD_FORMAT;
   if (!k_ok(M.format, k)) return MOE_ERR_BAD_FORMAT;
   if (!M.packed) return MOE_ERR_NULL_POINTER;
   if (!aligned(M.packed, 16)) return MOE_ERR_MISALIGNED;
@@ -88,6 +90,9 @@ int check_matrix(const moe_matrix& M, int n, int k, int E, MatDev* out) {
   } else if (M.format == MOE_FMT_MXFP4) {
     if (!M.scales) return MOE_ERR_NULL_POINTER;
     scale_bytes = (size_t)n * (k / 32);
+  } else if (M.format == MOE_FMT_FP8_E4M3) {
+    if (!M.tensor_scale) return MOE_ERR_NULL_POINTER;
+    if (!aligned(M.tensor_scale, 4)) return MOE_ERR_MISALIGNED;
   }
   const int64_t salign = M.format == MOE_FMT_MXFP4 ? 1 : 2;  // scale element bytes
   if (scale_bytes && E > 1 && (M.scale_stride < (int64_t)scale_bytes || M.scale_stride % salign))
@@ -197,7 +202,8 @@ cudaError_t launch_gate_up(int fmt, int rb, int grid, size_t smem, cudaStream_t 
     case MOE_FMT_Q4_AFFINE_G64:
       return launch_gate_up_fmt<MOE_FMT_Q4_AFFINE_G64, XBF16>(rb, grid, smem, st, p);
     case MOE_FMT_NVFP4: return launch_gate_up_fmt<MOE_FMT_NVFP4, XBF16>(rb, grid, smem, st, p);
-    default: return launch_gate_up_fmt<MOE_FMT_MXFP4, XBF16>(rb, grid, smem, st, p);
+    case MOE_FMT_MXFP4: return launch_gate_up_fmt<MOE_FMT_MXFP4, XBF16>(rb, grid, smem, st, p);
+    default: return launch_gate_up_fmt<MOE_FMT_FP8_E4M3, XBF16>(rb, grid, smem, st, p);
   }
 }
 
@@ -217,7 +223,8 @@ cudaError_t launch_down(int fmt, int rb, int grid, size_t smem, cudaStream_t st,
     case MOE_FMT_BF16: return launch_down_fmt<MOE_FMT_BF16>(rb, grid, smem, st, p);
     case MOE_FMT_Q4_AFFINE_G64: return launch_down_fmt<MOE_FMT_Q4_AFFINE_G64>(rb, grid, smem, st, p);
     case MOE_FMT_NVFP4: return launch_down_fmt<MOE_FMT_NVFP4>(rb, grid, smem, st, p);
-    default: return launch_down_fmt<MOE_FMT_MXFP4>(rb, grid, smem, st, p);
+    case MOE_FMT_MXFP4: return launch_down_fmt<MOE_FMT_MXFP4>(rb, grid, smem, st, p);
+    default: return launch_down_fmt<MOE_FMT_FP8_E4M3>(rb, grid, smem, st, p);
   }
 }
 
@@ -271,8 +278,7 @@ bool plan_fused(const moe_cfg& c, int m, bool has_shared, int fmt, int sms, Fuse
   if (off > kFusedSmemBudget) return false;
   // down-row tile: as many phase-E slots (column block of one expert's down rows, with their
   // scale rows) as the rest of the budget holds, up to every slot a call can have
-  const size_t prb = fmt == MOE_FMT_F32 ? (size_t)kmax * 4
-                     : fmt == MOE_FMT_BF16 ? (size_t)kmax * 2 : (size_t)kmax / 2;
+  const size_t prb = packed_row_bytes(fmt, kmax);
   const size_t srb = q4 ? (size_t)(kmax / 64) * 2
                      : fmt == MOE_FMT_NVFP4 ? (size_t)(kmax / 16)
                      : fmt == MOE_FMT_MXFP4 ? (size_t)(kmax / 32) : 0;
@@ -345,7 +351,7 @@ cudaError_t launch_fused_rb(int m, const Params& p, const FusedPlan& fp, cudaStr
 bool fused_formats_ok(int fmt, bool xbf16) {
   return (fmt == MOE_FMT_F32 && !xbf16) ||
          (xbf16 && (fmt == MOE_FMT_BF16 || fmt == MOE_FMT_Q4_AFFINE_G64 ||
-                    fmt == MOE_FMT_NVFP4 || fmt == MOE_FMT_MXFP4));
+                    fmt == MOE_FMT_NVFP4 || fmt == MOE_FMT_MXFP4 || fmt == MOE_FMT_FP8_E4M3));
 }
 
 cudaError_t launch_fused(int fmt, bool xbf16, int m, const Params& p, const FusedPlan& fp,
@@ -355,7 +361,8 @@ cudaError_t launch_fused(int fmt, bool xbf16, int m, const Params& p, const Fuse
     case MOE_FMT_BF16: return launch_fused_rb<MOE_FMT_BF16, true>(m, p, fp, st);
     case MOE_FMT_Q4_AFFINE_G64: return launch_fused_rb<MOE_FMT_Q4_AFFINE_G64, true>(m, p, fp, st);
     case MOE_FMT_NVFP4: return launch_fused_rb<MOE_FMT_NVFP4, true>(m, p, fp, st);
-    default: return launch_fused_rb<MOE_FMT_MXFP4, true>(m, p, fp, st);
+    case MOE_FMT_MXFP4: return launch_fused_rb<MOE_FMT_MXFP4, true>(m, p, fp, st);
+    default: return launch_fused_rb<MOE_FMT_FP8_E4M3, true>(m, p, fp, st);
   }
 }
 
@@ -440,6 +447,7 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
   p.before_ffn = c.weight_before_ffn;
   p.shared_kind = c.shared_kind;
   p.out_bf16 = c.out_dtype == MOE_FMT_BF16;
+  p.act_kind = c.activation;
   p.rsf = c.routed_scaling_factor;
   const int te = m * c.top_k;
   p.cap = te < c.num_experts ? te : c.num_experts;
@@ -618,4 +626,4 @@ extern "C" const char* moe_status_string(int status) {
 
 extern "C" int moe_last_cuda_error(void) { return g_last_cuda_error; }
 
-extern "C" int moe_version(void) { return 100; }
+extern "C" int moe_version(void) { return 200; }

@@ -87,7 +87,7 @@ inline WsLayout make_layout(int m, int h, int E, int k, int I, int S, int n_tile
 
 struct Params {
   int m, h, E, k, I, S;
-  int routing, norm, raw, has_bias, before_ffn, shared_kind, out_bf16;
+  int routing, norm, raw, has_bias, before_ffn, shared_kind, out_bf16, act_kind;
   float rsf;
   int cap;             // min(m*k, E): routed work slots
   int n_tiles_i;       // routed gate/up tiles per expert
@@ -152,6 +152,17 @@ __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v &
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + __expf(-z)); }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+// GELU, tanh form, times u: g/2 * (1 + tanh(sqrt(2/pi) * (g + 0.044715 g^3))) * u.
+__device__ __forceinline__ float gelu_tanh_mul(float g, float u) {
+  const float t = tanhf(0.7978845608028654f * fmaf(0.044715f * g, g * g, g));
+  return 0.5f * g * (1.0f + t) * u;
+}
+
+// The expert activation of the call: SwiGLU or GeGLU (moe_activation).
+__device__ __forceinline__ float act_mul(int act, float g, float u) {
+  return act == MOE_ACT_GEGLU ? gelu_tanh_mul(g, u) : silu_mul(g, u);
+}
 
 // Optional phase timestamps (build with -DMOE_PHASE_TIMERS): thread 0 of every CTA records
 // the SM cycle counter at each phase boundary into the (otherwise unused) down-partials region

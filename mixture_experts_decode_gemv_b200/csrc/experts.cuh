@@ -29,9 +29,13 @@ template <> struct Fmt<MOE_FMT_BF16> { static constexpr int kElems = 8; };
 template <> struct Fmt<MOE_FMT_Q4_AFFINE_G64> { static constexpr int kElems = 32; };
 template <> struct Fmt<MOE_FMT_NVFP4> { static constexpr int kElems = 32; };
 template <> struct Fmt<MOE_FMT_MXFP4> { static constexpr int kElems = 32; };
+template <> struct Fmt<MOE_FMT_FP8_E4M3> { static constexpr int kElems = 16; };
 
 __host__ __device__ constexpr size_t packed_row_bytes(int fmt, int k) {
-  return fmt == MOE_FMT_F32 ? (size_t)k * 4 : fmt == MOE_FMT_BF16 ? (size_t)k * 2 : (size_t)k / 2;
+  return fmt == MOE_FMT_F32 ? (size_t)k * 4
+         : fmt == MOE_FMT_BF16 ? (size_t)k * 2
+         : fmt == MOE_FMT_FP8_E4M3 ? (size_t)k
+                                   : (size_t)k / 2;
 }
 
 // One decoded 16-byte chunk of a weight row. For the 4-bit affine format the codes are kept as
@@ -43,6 +47,7 @@ template <> struct Dec<MOE_FMT_BF16> { float w[8]; };
 template <> struct Dec<MOE_FMT_Q4_AFFINE_G64> { float f[32]; float s16, bm; };
 template <> struct Dec<MOE_FMT_NVFP4> { float v[32]; float s0, s1; };
 template <> struct Dec<MOE_FMT_MXFP4> { float v[32]; float s; };
+template <> struct Dec<MOE_FMT_FP8_E4M3> { float w[16]; };
 
 // Row-local pointers of one weight row of one expert matrix.
 struct RowRef {
@@ -67,6 +72,8 @@ __device__ __forceinline__ RowRef row_ref(const MatDev& M, int e, int row) {
     r.ts = __ldg(M.tscale + e);
   } else if constexpr (FMT == MOE_FMT_MXFP4) {
     r.sc = M.scales + (size_t)e * M.sstride + (size_t)row * (M.k / 32);
+  } else if constexpr (FMT == MOE_FMT_FP8_E4M3) {
+    r.ts = __ldg(M.tscale + e);
   }
   return r;
 }
@@ -167,6 +174,17 @@ __device__ __forceinline__ void decode(const Chunk& ch, Dec<FMT>& d) {
   } else if constexpr (FMT == MOE_FMT_MXFP4) {
     decode_e2m1x32(q, d.v);
     d.s = e8m0_to_float(ch.aux & 0xFFu);
+  } else if constexpr (FMT == MOE_FMT_FP8_E4M3) {  // byte j is element j
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+            (__nv_fp8x2_storage_t)((q[t] >> (16 * b)) & 0xFFFFu), __NV_E4M3);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+        d.w[4 * t + 2 * b] = f.x;
+        d.w[4 * t + 2 * b + 1] = f.y;
+      }
   } else {  // NVFP4
     decode_e2m1x32(q, d.v);
     const __half2_raw hs =
@@ -186,6 +204,8 @@ template <int FMT>
 __device__ __forceinline__ int x_quad(int q) {  // logical quad -> stored quad
   if constexpr (FMT == MOE_FMT_Q4_AFFINE_G64 || FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_MXFP4) {
     return (q & ~7) | ((q ^ (q >> 3)) & 7);                // 8 quads per chunk
+  } else if constexpr (FMT == MOE_FMT_FP8_E4M3) {
+    return (q & ~3) | ((q ^ (q >> 3)) & 3);                // 4 quads per chunk
   } else if constexpr (FMT == MOE_FMT_BF16) {
     return (q & ~1) | ((q ^ (q >> 3)) & 1);                // 2 quads per chunk
   } else {
@@ -203,7 +223,7 @@ __device__ __forceinline__ float4 x_load(const float* row, int q) {
 template <int FMT>
 __device__ __forceinline__ float dot(const Dec<FMT>& d, const float* row, int c, float xsum) {
   constexpr int kQ = Fmt<FMT>::kElems / 4;  // quads per chunk
-  if constexpr (FMT == MOE_FMT_F32 || FMT == MOE_FMT_BF16) {
+  if constexpr (FMT == MOE_FMT_F32 || FMT == MOE_FMT_BF16 || FMT == MOE_FMT_FP8_E4M3) {
     float a = 0.f;
 #pragma unroll
     for (int i = 0; i < kQ; ++i) {
@@ -538,7 +558,7 @@ __global__ void __launch_bounds__(kThreads) gate_up_swiglu_kernel(const __grid_c
             u *= w;
           }
         }
-        dst[pos * N + i] = silu_mul(g, u);
+        dst[pos * N + i] = act_mul(p.act_kind, g, u);
       }
     }
     __syncthreads();

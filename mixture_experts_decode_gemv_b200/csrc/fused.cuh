@@ -180,7 +180,7 @@ struct FusedRoute {
   int slot_n[kFusedMaxPairs];     // its number of pairs
   int n_active;
   float bias[MOE_MAX_EXPERTS];    // expert biases, staged once per call
-  float ts[kFusedMaxPairs + 1];   // NVFP4 tensor scale of each phase-E slot's down matrix
+  float ts[kFusedMaxPairs + 1];   // NVFP4 / FP8 tensor scale of each phase-E slot's down matrix
 };
 
 // Route row r (one warp) into the CTA's shared routing tables (same rule and arithmetic as the
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
             g = ag[j];
             u = au[j];
           }
-        p.act_sh[(size_t)lane * p.S + i] = silu_mul(g * A.ts, u * B.ts);
+        p.act_sh[(size_t)lane * p.S + i] = act_mul(p.act_kind, g * A.ts, u * B.ts);
       }
     }
   }
@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
                                 ? D.biases + (size_t)e * D.sstride + (size_t)c0 * srb
                                 : nullptr;
       const unsigned wb = (unsigned)(ncols * prb), sb = (unsigned)(ncols * srb);
-      if (FMT == MOE_FMT_NVFP4) R.ts[sl] = __ldg(D.tscale + e);
+      if (FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_FP8_E4M3) R.ts[sl] = __ldg(D.tscale + e);
       bool in_tile = false;
       if (sl < s_tile_n) {
         in_tile = sb % 16 == 0 && ((uintptr_t)ssrc | (uintptr_t)bsrc) % 16 == 0;
@@ -496,7 +496,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
           g *= w;
           u *= w;
         }
-        p.act[(size_t)(beg + lane) * p.I + i] = silu_mul(g, u);
+        p.act[(size_t)(beg + lane) * p.I + i] = act_mul(p.act_kind, g, u);
       }
     }
   }
@@ -564,7 +564,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
         const int cr = col + min(r, nvalid - 1);
         A[r] = in_tile ? tile_row_ref<FMT>(D, e, sl, K, fp, cr - c0) : row_ref<FMT>(D, e, cr);
       }
-      const float ts = FMT == MOE_FMT_NVFP4 ? R.ts[slot] : 1.f;
+      const float ts = (FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_FP8_E4M3) ? R.ts[slot] : 1.f;
       float acc[NR][RB];
       rowsN_dot<FMT, RB, kPlain, NR>(A, nch, xr, xsr, n, acc);
       if (lane < n) {

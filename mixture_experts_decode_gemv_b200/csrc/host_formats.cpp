@@ -131,6 +131,9 @@ extern "C" int moe_packed_bytes(int format, int n, int k, size_t* packed, size_t
     case MOE_FMT_MXFP4:
       if (k % 32) return MOE_ERR_BAD_SHAPE;
       *packed = nk / 2; *scales = nk / 32; *biases = 0; return MOE_OK;
+    case MOE_FMT_FP8_E4M3:
+      if (k % 16) return MOE_ERR_BAD_SHAPE;
+      *packed = nk; *scales = 0; *biases = 0; return MOE_OK;
     default: return MOE_ERR_BAD_FORMAT;
   }
 }
@@ -232,6 +235,19 @@ extern "C" int moe_quantize_mxfp4(const float* w, int n, int k, uint8_t* packed,
   return MOE_OK;
 }
 
+extern "C" int moe_quantize_fp8_e4m3(const float* w, int n, int k, uint8_t* packed,
+                                     float* tensor_scale) {
+  if (!w || !packed || !tensor_scale) return MOE_ERR_NULL_POINTER;
+  if (n <= 0 || k <= 0 || k % 16) return MOE_ERR_BAD_SHAPE;
+  const size_t nk = (size_t)n * k;
+  double amax = 0.0;
+  for (size_t i = 0; i < nk; ++i) amax = std::max(amax, std::fabs((double)w[i]));
+  const float ts = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
+  *tensor_scale = ts;
+  for (size_t i = 0; i < nk; ++i) packed[i] = f64_to_e4m3((double)w[i] / (double)ts);
+  return MOE_OK;
+}
+
 extern "C" int moe_dequantize(int format, const void* packed, const void* scales,
                               const void* biases, const float* tensor_scale, int n, int k,
                               float* out) {
@@ -289,6 +305,14 @@ extern "C" int moe_dequantize(int format, const void* packed, const void* scales
           const double sc = e8m0_to_double(s[(size_t)r * (k / 32) + j / 32]);
           out[(size_t)r * k + j] = (float)(e2m1_to_double(c) * sc);
         }
+      return MOE_OK;
+    }
+    case MOE_FMT_FP8_E4M3: {
+      if (!tensor_scale) return MOE_ERR_NULL_POINTER;
+      if (k % 16) return MOE_ERR_BAD_SHAPE;
+      const uint8_t* p = (const uint8_t*)packed;
+      const double ts = (double)tensor_scale[0];
+      for (size_t i = 0; i < nk; ++i) out[i] = (float)(e4m3_to_double(p[i]) * ts);
       return MOE_OK;
     }
     default:

@@ -81,6 +81,13 @@ __device__ __forceinline__ uint32_t key_bits(float v) {
 // a selection round is one warp max over the lanes' heads and a ballot of the lanes holding it
 // (a second reduction, min id, only when several lanes tie), after which the winning lane pops
 // its head. Returns false when a selected key is not a finite number.
+// Score of the non-softmax routers: sigmoid(l), or sqrt(softplus(l)) with
+// softplus(l) = max(l, 0) + log1p(e^-|l|) (no overflow for large |l|).
+__device__ __forceinline__ float router_score(int routing, float l) {
+  if (routing == MOE_ROUTE_SQRTSOFTPLUS) return sqrtf(fmaxf(l, 0.f) + log1pf(expf(-fabsf(l))));
+  return 1.0f / (1.0f + expf(-l));
+}
+
 // The routing options of a call, copied out of the kernel parameters into registers (a routine
 // that reads them through a reference to the parameter block would load each one from memory).
 struct RouteCfg {
@@ -128,7 +135,7 @@ __device__ __forceinline__ bool route_row_nj(const RouteCfg& c, int r, const flo
   const int lane = threadIdx.x & 31;
   const int E = c.E, k = c.k;
   const float* lrow = c.logits + (size_t)r * (E + 1);
-  const bool sig_keys = c.routing == MOE_ROUTE_SIGMOID && !c.raw;
+  const bool sig_keys = c.routing != MOE_ROUTE_SOFTMAX && !c.raw;  // keys are router scores
   const bool add_bias = sig_keys && c.has_bias;
   const bool gated = c.gated;
   float lg[NJ], bs[NJ];
@@ -147,7 +154,7 @@ __device__ __forceinline__ bool route_row_nj(const RouteCfg& c, int r, const flo
     const int e = lane + 32 * j;
     float kv = lg[j];
     if (sig_keys) {
-      kv = 1.0f / (1.0f + expf(-lg[j]));
+      kv = router_score(c.routing, lg[j]);
       if (add_bias) kv += bs[j];
     }
     key[j] = e < E ? key_bits(kv) : 0u;  // a real key is >= key_bits(-inf) > 0
@@ -222,7 +229,7 @@ __device__ __forceinline__ bool route_row_nj(const RouteCfg& c, int r, const flo
     wv = expf(my_l - top_l);
     if (!c.norm) wv = wv / warp_sum(den);
   } else {
-    wv = 1.0f / (1.0f + expf(-my_l));
+    wv = router_score(c.routing, my_l);
   }
   if (lane >= k) wv = 0.f;
   if (c.norm) {

@@ -32,6 +32,7 @@ def make_cfg(cfg: LayerConfig, out_dtype: str = "f32") -> B.moe_cfg:
     c.shared_kind = B.SHARED_CODES[cfg.shared_kind] if cfg.has_shared else B.MOE_SHARED_NONE
     c.x_dtype = B.FORMAT_CODES[cfg.x_dtype]
     c.out_dtype = B.FORMAT_CODES[out_dtype]
+    c.activation = B.ACTIVATION_CODES[cfg.activation]
     return c
 
 

@@ -121,9 +121,13 @@ LLAMA4_SCOUT = LayerConfig(
 QWEN3_30B_A3B_MXFP4 = QWEN3_30B_A3B.replace(name="qwen3_30b_a3b_mxfp4", fmt="mxfp4",
                                            m_list=(1, 4), index=5)
 
+# FP8 (E4M3, one scale per expert matrix) experts on the same shape: the pages' FP8 grouped decode.
+QWEN3_30B_A3B_FP8 = QWEN3_30B_A3B.replace(name="qwen3_30b_a3b_fp8", fmt="fp8_e4m3",
+                                         m_list=(1, 4), index=6)
+
 CONFIGS: Dict[str, LayerConfig] = {
     c.name: c for c in (TINY, QWEN3_30B_A3B, LFM2_8B_A1B, QWEN3_6_35B_A3B, LLAMA4_SCOUT,
-                        QWEN3_30B_A3B_MXFP4)
+                        QWEN3_30B_A3B_MXFP4, QWEN3_30B_A3B_FP8)
 }
 
 

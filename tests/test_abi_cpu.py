@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_status_strings():
-    assert B.moe_version() == 100
+    assert B.moe_version() == 200
     for st in range(-10, 1):
         assert B.moe_status_string(st) != "unknown status"
     assert B.moe_status_string(-99) == "unknown status"
@@ -244,6 +244,37 @@ def test_mxfp4_quantiser_round_trip_bound():
     lib_dec = B.moe_dequantize(B.MOE_FMT_MXFP4, packed, scales, None, None, n, k)
     np.testing.assert_array_equal(lib_dec, dec.astype(np.float32))
     assert B.moe_packed_bytes(B.MOE_FMT_MXFP4, 10, 128) == (640, 40, 0)
+
+
+def test_fp8_quantiser_round_trip_bound():
+    rng = np.random.default_rng(5)
+    n, k = 8, 64
+    w = (rng.standard_normal((n, k)) * 0.05).astype(np.float32)
+    packed, ts = B.moe_quantize_fp8_e4m3(w)
+    assert ts[0] == np.float32(np.abs(w.astype(np.float64)).max() / 448.0)
+    from mixture_experts_decode_gemv_b200.synthetic import MatrixSlab
+    dec = ref.decode_matrix(MatrixSlab("fp8_e4m3", n, k, packed[None], tensor_scale=ts), 0)
+    v = w.astype(np.float64) / float(ts[0])
+    # E4M3 has 3 mantissa bits: a normal value is within 2^-4 relative of its code; below 2^-6
+    # the subnormal step is 2^-9
+    err = np.abs(dec / float(ts[0]) - v)
+    assert np.all(err <= np.maximum(np.abs(v) * 2.0 ** -4, 2.0 ** -10) + 1e-12)
+    lib_dec = B.moe_dequantize(B.MOE_FMT_FP8_E4M3, packed, None, None, ts, n, k)
+    np.testing.assert_array_equal(lib_dec, dec.astype(np.float32))
+    assert B.moe_packed_bytes(B.MOE_FMT_FP8_E4M3, 10, 64) == (640, 0, 0)
+
+
+def test_new_options_are_refused_out_of_range():
+    c = _small_cfg()
+    c.activation = 2
+    assert _call(c) == B.MOE_ERR_BAD_OPTION
+    c = _small_cfg()
+    c.routing = 3
+    assert _call(c) == B.MOE_ERR_BAD_OPTION
+    c = _small_cfg(routing="sqrtsoftplus", has_expert_bias=True)
+    assert _call(c) == B.MOE_ERR_NULL_POINTER         # bias required, as for sigmoid
+    t = _fake_table(fmt=B.MOE_FMT_FP8_E4M3)
+    assert _call(_small_cfg(), routed=t) == B.MOE_ERR_NULL_POINTER  # fp8 needs its scales
 
 
 def test_dequantize_bf16_and_f32_plain():

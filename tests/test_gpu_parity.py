@@ -45,6 +45,16 @@ SMALL = {
                                 moe_inter=96, shared_inter=64, shared_kind="plain", fmt="mxfp4",
                                 routing="sigmoid", has_expert_bias=True,
                                 routed_scaling_factor=1.5, index=208),
+    "ragged_fp8_geglu": LayerConfig(name="ragged_fp8_geglu", hidden=112, num_experts=7, top_k=3,
+                                    moe_inter=80, shared_inter=48, shared_kind="sigmoid_gate",
+                                    fmt="fp8_e4m3", activation="geglu", index=209),
+    "sqrtsoftplus_bias": LayerConfig(name="sqrtsoftplus_bias", hidden=128, num_experts=24,
+                                     top_k=4, moe_inter=64, fmt="bf16", routing="sqrtsoftplus",
+                                     has_expert_bias=True, routed_scaling_factor=2.5, index=210),
+    "sqrtsoftplus_geglu_q4": LayerConfig(name="sqrtsoftplus_geglu_q4", hidden=192,
+                                         num_experts=40, top_k=6, moe_inter=128,
+                                         fmt="q4_affine_g64", routing="sqrtsoftplus",
+                                         norm_topk_prob=False, activation="geglu", index=211),
 }
 
 _CACHE = {}
@@ -225,7 +235,7 @@ class _Path:
 
 
 PATH_CASES = [(n, m) for n in ("qwen3_30b_a3b", "lfm2_8b_a1b", "qwen3_6_35b_a3b", "llama4_scout",
-                                "qwen3_30b_a3b_mxfp4")
+                                "qwen3_30b_a3b_mxfp4", "qwen3_30b_a3b_fp8")
               for m in (1, 2, 3, 4)] + [(n, m) for n in SMALL for m in (1, 4)]
 
 
