@@ -39,7 +39,7 @@ METRIC = "MoE decode layer µs and tokens/s at m=1..64; achieved HBM GB/s vs B20
 # dram__bytes_write.sum, one ncu capture of the current kernel; see profiles/). Keyed by
 # (workload config name, m, launches per call); absent keys report null.
 PROFILED_TRAFFIC = {
-    ("qwen3_30b_a3b", 1, 1): 77.5e6,  # profiles/moe_fused_kernel_qwen3_30b_a3b_m1.md
+    ("qwen3_30b_a3b", 1, 1): 77.6e6,  # profiles/moe_fused_kernel_qwen3_30b_a3b_m1.md
 }
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -146,12 +146,13 @@ def dist_setup():
     return ws, rank, local
 
 
-def max_over_ranks(v: float, ws: int) -> float:
+def max_over_ranks(v: float, ws: int, device: str = "cuda") -> float:
+    """The largest of the ranks' values (a rank's timed milliseconds): the job's time."""
     if ws == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
