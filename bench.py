@@ -57,6 +57,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--cold-steps", type=int, default=50,
+                    help="calls timed one by one after an L2 flush (0: skip)")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--path", choices=("auto", "chain"), default="auto",
                     help="launch path: automatic (persistent kernel for m <= 4) or the chain")
@@ -343,6 +345,26 @@ def run_ours(args, cfg):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), wsz)
 
+    # cold variant: L2 flushed (a write of twice its size) before every call, each call timed
+    # on its own; the median is reported beside the rotating-replica figure
+    cold_n = min(args.cold_steps, steps)
+    cold_us = None
+    if cold_n > 0:
+        flush = torch.empty(2 * l2, dtype=torch.uint8, device=f"cuda:{dev_index}")
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(cold_n)]
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for j, (a, b) in enumerate(evs):
+                flush.fill_(j & 0xFF)
+                a.record(stream)
+                reps[j % R].forward(xs[j % nx], out, ws, stream=stream)
+                b.record(stream)
+        torch.cuda.synchronize()
+        cold_us = 1000.0 * statistics.median([a.elapsed_time(b) for a, b in evs])
+        cold_us = 1000.0 * max_over_ranks(cold_us / 1000.0, wsz)
+        del flush
+
     kernels_per_step = dev0.launches(m)
     kernel_name = ("moe_fused_kernel (whole layer, one persistent launch)" if kernels_per_step == 1
                    else "whole layer (router_topk_group + gate_up_swiglu + down_blend, PDL)")
@@ -381,6 +403,10 @@ def run_ours(args, cfg):
                 "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": e2e_steps},
         "gpu_launches": kernels_per_step * steps,
         "clocks": clk,
+        "cold": None if cold_us is None else {
+            "us_per_layer_median": cold_us, "steps": cold_n,
+            "policy": "L2 flushed by a write of 2x its size before every call; each call timed "
+                      "alone with CUDA events; median"},
         "device_status": status,
     }
     if rank == 0 and wsz == 1 and not args.no_cpu_baseline:
