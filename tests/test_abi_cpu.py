@@ -35,6 +35,26 @@ def test_library_exports_every_declared_symbol():
     assert set(names) == set(B.EXPORTS)
 
 
+def test_header_enum_values_match_the_binding():
+    import re
+    with open(os.path.join(os.path.dirname(B.LIB_PATH), "..", "include", "moe_decode.h")) as f:
+        text = f.read()
+    vals = {k: int(v) for k, v in re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(-?\d+)", text)}
+    checked = 0
+    for name, v in vals.items():
+        if hasattr(B, name):
+            assert getattr(B, name) == v, name
+            checked += 1
+    assert checked >= 20, checked
+    # every format, routing and activation the Python side names exists in the header
+    for table in (B.FORMAT_CODES, B.ROUTING_CODES, B.ACTIVATION_CODES, B.SHARED_CODES):
+        assert set(table.values()) <= set(vals.values())
+    # the struct layout the binding passes has the header's field count and order
+    fields = re.search(r"typedef struct moe_cfg \{(.*?)\} moe_cfg;", text, re.S).group(1)
+    names = re.findall(r"(?:int32_t|float)\s+(\w+);", fields)
+    assert names == [f[0] for f in B.moe_cfg._fields_]
+
+
 def test_version_and_status_strings():
     assert B.moe_version() == 200
     for st in range(-10, 1):
