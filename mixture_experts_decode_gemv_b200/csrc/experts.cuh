@@ -3,12 +3,13 @@
 // Every weight row is reduced by one whole warp: lane l takes the row's 16-byte chunks l, l+32,
 // l+64, ... in order, decodes each in registers and accumulates in fp32, then a butterfly warp
 // sum finishes the row. The same arithmetic runs whether the chunks are streamed from global
-// memory (non-allocating 128-bit loads) or from a shared-memory ring, so both launch paths give
-// identical bits. Activation rows are staged once in shared memory as fp32.
+// memory (non-allocating 128-bit loads, L2 evict-first) or read with plain loads from a
+// shared-memory tile, so both launch paths give identical bits. Activation rows are staged once
+// in shared memory as fp32.
 //
 // gate_up_swiglu_kernel: one CTA = 32 (gate_i, up_i) row pairs of one active expert (or of the
 //   shared expert), 4 per warp, for every pair routed to that expert; act[pos, i] = silu(g) * u
-//   per sorted pair position.
+//   (or gelu(g) * u) per sorted pair position.
 // down_blend_kernel: one CTA = 64 output columns of one active expert's down matrix (or the
 //   shared expert's), 8 per warp taken two at a time, for every row that uses it, into per-pair
 //   partials; the CTA that completes a column tile last (atomic ticket, no spinning) blends the

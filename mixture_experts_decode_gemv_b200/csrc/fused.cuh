@@ -4,19 +4,21 @@
 //   A  router logits: stage the m activation rows in shared memory as fp32, one warp per
 //      (router row, activation row) dot product (router rows were asked into L2 before the
 //      programmatic-launch wait); arrive at grid barrier 1 without waiting.
-//   B  shared expert gate+up (needs no routing): this CTA's slice of the S row pairs.
+//   B  shared expert gate+up (needs no routing): this CTA's slice of the S row pairs. Meanwhile
+//      one idle warp runs the routing code on throw-away rows, so its instructions are cached
+//      when phase C needs them.
 //   C  wait at barrier 1; every CTA routes every row and groups the pairs by expert in its own
 //      shared memory (m*k <= 32 pairs).
 //   D  routed gate+up: the U*I row pairs of the U active experts in equal contiguous slices, one
-//      per CTA; first the CTA asks L2 for the down rows it will need in phase E (when the whole
-//      call's down rows fit comfortably in L2), so they arrive while gate/up streams. Arrive and
-//      wait at grid barrier 2.
+//      per CTA. The last warp bulk-copies the down rows this CTA needs in phase E into a
+//      shared-memory tile (slots that do not fit are asked into L2 instead), so they arrive
+//      while gate/up streams. Arrive and wait at grid barrier 2.
 //   E  down + blend: each CTA owns a contiguous range of output columns for all rows; y for each
-//      (column, active expert) and for the shared expert, then the blend: routed slots in slot
-//      order times their weight, then gamma times the shared expert. No atomics.
+//      (column, active expert) and for the shared expert, from the tile, then the blend: routed
+//      slots in slot order times their weight, then gamma times the shared expert. No atomics.
 // Every weight row is reduced by one warp with the multi-kernel path's arithmetic (lane l takes
 // chunks l, l+32, ..., then a butterfly sum), so both paths give the same bits and a row's bits
-// do not depend on m. Each grid-barrier wait is bounded (clock64 budget): on expiry it records
+// do not depend on m. Every wait is bounded (clock64 budget): on expiry it records
 // MOE_ERR_DEVICE_TIMEOUT in the workspace status word and carries on, so the kernel terminates.
 #pragma once
 
