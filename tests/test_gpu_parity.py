@@ -55,6 +55,18 @@ SMALL = {
                                          num_experts=40, top_k=6, moe_inter=128,
                                          fmt="q4_affine_g64", routing="sqrtsoftplus",
                                          norm_topk_prob=False, activation="geglu", index=211),
+    # hidden sizes that the chain's tensor-core gate/up tiles take (k-tiles of 4 chunks)
+    "mma_fp8_geglu": LayerConfig(name="mma_fp8_geglu", hidden=128, num_experts=10, top_k=3,
+                                 moe_inter=48, shared_inter=32, shared_kind="sigmoid_gate",
+                                 fmt="fp8_e4m3", activation="geglu", index=212),
+    "mma_mxfp4_bias": LayerConfig(name="mma_mxfp4_bias", hidden=256, num_experts=12, top_k=4,
+                                  moe_inter=64, fmt="mxfp4", routing="sigmoid",
+                                  has_expert_bias=True, index=213),
+    "mma_bf16_ragged_rows": LayerConfig(name="mma_bf16_ragged_rows", hidden=64, num_experts=6,
+                                        top_k=2, moe_inter=40, shared_inter=24,
+                                        shared_kind="plain", fmt="bf16", weight_before_ffn=True,
+                                        routing="sigmoid", select_on_raw_logits=True,
+                                        norm_topk_prob=False, index=214),
 }
 
 _CACHE = {}
@@ -134,13 +146,28 @@ def test_published_shapes_match_oracle(name, m):
     check_out(got if rows is None else got[rows], want)
 
 
-@pytest.mark.parametrize("name", ["ragged_nvfp4_gate", "ragged_q4_shared", "before_ffn_small"])
+def _mma_chain(cfg) -> bool:
+    """Whether chain calls of this layer may run gate/up on the tensor-core tiles."""
+    kelems = {"bf16": 8, "fp8_e4m3": 16, "nvfp4": 32, "mxfp4": 32}.get(cfg.fmt)
+    return kelems is not None and cfg.x_dtype == "bf16" and cfg.hidden % (4 * kelems) == 0
+
+
+@pytest.mark.parametrize("name", ["ragged_nvfp4_gate", "ragged_q4_shared", "before_ffn_small",
+                                  "mma_fp8_geglu", "mma_mxfp4_bias"])
 def test_rows_do_not_depend_on_m(name):
+    # Within one launch path a row's bits do not depend on the other rows. Calls of m <= 4 take
+    # the persistent kernel; larger ones the chain, whose gate/up may run on tensor-core tiles
+    # (a different order of the fp32 sums): those rows agree with m = 1 within the tolerance.
     lay, dev, _ = layer_for(SMALL[name])
     full, _, _ = run(dev, lay.x(64))
-    for r in (0, 9, 63):
+    for r in (0, 9, 59):
+        part, _, _ = run(dev, lay.x(5, offset=r))
+        np.testing.assert_array_equal(part, full[r:r + 5])
         one, _, _ = run(dev, lay.x(1, offset=r))
-        np.testing.assert_array_equal(one[0], full[r])
+        if _mma_chain(dev.cfg):
+            check_out(one[0], full[r].astype(np.float64))
+        else:
+            np.testing.assert_array_equal(one[0], full[r])
 
 
 def test_repeated_calls_are_bit_identical_and_workspace_reusable():
@@ -153,9 +180,11 @@ def test_repeated_calls_are_bit_identical_and_workspace_reusable():
         dev.forward(x, out, ws)
         outs.append(out.cpu())
     torch.cuda.synchronize()
-    assert torch.equal(outs[0], outs[2]) and torch.equal(outs[0], outs[4])
-    assert torch.equal(outs[1][0], outs[0][0])
-    assert torch.equal(outs[3], outs[0][:4])
+    assert torch.equal(outs[0], outs[2]) and torch.equal(outs[0], outs[4])   # same path, same bits
+    assert torch.equal(outs[1][0], outs[3][0])                               # m = 1 and 4: one kernel
+    # m = 8 takes the chain (tensor-core gate/up): the same rows within the tolerance
+    check_out(outs[1][0].numpy(), outs[0][0].double().numpy())
+    check_out(outs[3].numpy(), outs[0][:4].double().numpy())
     assert dev.device_status(ws) == B.MOE_OK
 
 
@@ -291,3 +320,21 @@ def test_grid_barrier_timeout_is_reported_and_the_workspace_recovers():
     torch.cuda.synchronize()
     assert dev.device_status(ws) == B.MOE_OK
     assert torch.equal(out, want)
+
+
+@pytest.mark.parametrize("name", ["max_experts", "mma_fp8_geglu", "mma_mxfp4_bias",
+                                  "mma_bf16_ragged_rows"])
+def test_tensor_core_and_cuda_core_gate_up_agree(name):
+    """The chain's two gate/up implementations on the same call, within the tolerance."""
+    import os
+    lay, dev, _ = layer_for(SMALL[name])
+    x = lay.x(33)
+    try:
+        os.environ["MOE_DECODE_MMA"] = "1"   # tensor-core tiles for every eligible format
+        tc, rt_a, _ = run(dev, x)
+        os.environ["MOE_DECODE_MMA"] = "0"   # CUDA-core tiles
+        cc, rt_b, _ = run(dev, x)
+    finally:
+        os.environ.pop("MOE_DECODE_MMA", None)
+    np.testing.assert_array_equal(rt_a["idx"], rt_b["idx"])
+    check_out(tc, cc.astype(np.float64))
