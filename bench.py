@@ -239,6 +239,8 @@ def run_ours(args, cfg):
     from mixture_experts_decode_gemv_b200.synthetic import POOL_ROWS, SyntheticLayer
 
     wsz, rank, local = dist_setup()
+    from mixture_experts_decode_gemv_b200 import binding as B
+    B.moe_debug_set_path(1 if args.path == "chain" else 0)
     dev_index = torch.cuda.current_device()
     m = args.m
     lay = SyntheticLayer(cfg)
@@ -423,8 +425,6 @@ def main():
     args = parse_args()
     from mixture_experts_decode_gemv_b200.synthetic import CONFIGS
     cfg = CONFIGS[args.config]
-    if args.path == "chain":
-        os.environ["MOE_DECODE_PATH"] = "chain"
     if args.m < 1 or args.m > 64:
         raise SystemExit("--m must be in 1..64")
     if args.impl == "reference":

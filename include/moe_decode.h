@@ -193,6 +193,13 @@ int moe_decode_launches(const moe_cfg* cfg, int m, const moe_expert_table* route
  * The decode pages have no counterpart. */
 int moe_debug_barrier_test(int extra_arrivals, long long spin_limit_cycles);
 
+/* Test aid: choose the launch path of every later forward call in this process. path 0 is the
+ * automatic choice; path 1 forces the multi-kernel path (router, gate/up, down launches) at any
+ * m, so tests can compare the two paths bit for bit on the same call. Process-wide; do not call
+ * it while other threads run forward calls. Returns MOE_ERR_BAD_OPTION for other values. The
+ * decode pages have no counterpart. */
+int moe_debug_set_path(int path);
+
 /* Copy the routing and grouping of the last forward call that used `workspace` to host arrays
  * (synchronises `stream`). Any output pointer may be NULL to skip it. Sizes: idx, weights,
  * sorted_pairs, token_to_perm: m*top_k; expert_offsets: num_experts+1; active: min(m*top_k, E);

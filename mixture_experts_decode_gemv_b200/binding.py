@@ -54,6 +54,7 @@ EXPORTS = (
     "moe_quantize_nvfp4", "moe_dequantize", "moe_status_string", "moe_last_cuda_error",
     "moe_version", "moe_decode_forward_no_alloc", "moe_decode_launches",
     "moe_debug_barrier_test", "moe_quantize_mxfp4", "moe_quantize_fp8_e4m3",
+    "moe_debug_set_path",
 )
 
 MOE_NO_ALLOC_SCRATCH_BYTES = 16 << 20
@@ -120,6 +121,7 @@ def _load() -> ctypes.CDLL:
         "moe_decode_launches": [P(moe_cfg), i32, P(moe_expert_table), P(moe_expert_table),
                                 P(ctypes.c_int32)],
         "moe_debug_barrier_test": [i32, i64],
+        "moe_debug_set_path": [i32],
         "moe_status_string": [i32],
         "moe_last_cuda_error": [],
         "moe_version": [],
@@ -211,6 +213,11 @@ def moe_decode_launches(cfg: moe_cfg, m: int, routed: moe_expert_table,
 def moe_debug_barrier_test(extra_arrivals: int, spin_limit_cycles: int) -> None:
     """Failure-detection test aid: make the persistent kernel's grid-barrier waits run out."""
     _check(lib.moe_debug_barrier_test(extra_arrivals, spin_limit_cycles), "moe_debug_barrier_test")
+
+
+def moe_debug_set_path(path: int) -> None:
+    """Test aid: 0 automatic launch path, 1 the multi-kernel path at every m (process-wide)."""
+    _check(lib.moe_debug_set_path(path), "moe_debug_set_path")
 
 
 def moe_decode_read_routing(cfg: moe_cfg, m: int, workspace, workspace_bytes: int, stream=None):

@@ -7,14 +7,14 @@
 #include <cstdio>
 #include <cstring>
 #include <atomic>
+#include <cstdlib>
 #include <mutex>
 
-#include <cstdlib>
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 #include "experts.cuh"
 #include "fused.cuh"
-#include "mma_tiles.cuh"
 #include "router.cuh"
 
 using namespace moe;
@@ -128,6 +128,33 @@ WsLayout layout_of(const moe_cfg* c, int m) {
                      n_tiles_c_of(c->hidden));
 }
 
+// NVTX range around a library call (visible in Nsight timelines; a few ns when no tool listens).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
+// One line on stderr the first time each (launch path, format, m) combination is dispatched,
+// when the environment variable MOE_DECODE_LOG is set to anything but "" or "0" (read once per
+// process; it changes nothing but this log).
+void log_dispatch_once(const char* path, int fmt, int m, int launches) {
+  static const bool on = [] {
+    const char* e = std::getenv("MOE_DECODE_LOG");
+    return e && *e && std::strcmp(e, "0") != 0;
+  }();
+  if (!on) return;
+  static std::mutex mu;
+  static unsigned long long seen[2][8] = {};  // bit m-1 of seen[path is chain][format]
+  std::lock_guard<std::mutex> lock(mu);
+  const int chain = path[0] == 'c';
+  unsigned long long& mask = seen[chain][fmt & 7];
+  const unsigned long long bit = 1ull << ((m - 1) & 63);
+  if (mask & bit) return;
+  mask |= bit;
+  std::fprintf(stderr, "[moe_decode] m=%d format=%d: %s (%d launch%s)\n", m, fmt, path, launches,
+               launches == 1 ? "" : "es");
+}
+
 // Compute capability 10.0 check, cached per device.
 int check_device() {
   static std::mutex mu;
@@ -170,54 +197,6 @@ cudaError_t launch(K kernel, int grid, int block, size_t smem, cudaStream_t st, 
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, p);
-}
-
-// Tensor-core gate/up tiles for chain calls: bf16 activations and bf16, FP8, NVFP4 or MXFP4
-// weights, k-tiles of four 16-byte chunks dividing h. By default only the 4-bit formats take
-// them (their CUDA-core tiles are bound by instruction issue at several rows per expert);
-// MOE_DECODE_MMA=1 extends them to bf16 and FP8, MOE_DECODE_MMA=0 turns them off (both for
-// comparisons).
-bool mma_gate_up_ok(int fmt, bool xbf16, int m, int h) {
-  const char* env = std::getenv("MOE_DECODE_MMA");
-  if (env && !std::strcmp(env, "0")) return false;
-  const bool all = env && !std::strcmp(env, "1");
-  if (!all && fmt != MOE_FMT_NVFP4 && fmt != MOE_FMT_MXFP4) return false;
-  int kelems = 0;
-  switch (fmt) {
-    case MOE_FMT_BF16: kelems = 8; break;
-    case MOE_FMT_FP8_E4M3: kelems = 16; break;
-    case MOE_FMT_NVFP4:
-    case MOE_FMT_MXFP4: kelems = 32; break;
-    default: return false;
-  }
-  return xbf16 && m > 4 && h % (4 * kelems) == 0;
-}
-
-// Blocks of 8 activation rows staged per pass of the tensor-core tiles (1, 2 or 4).
-int mma_blocks(int h, int m) {
-  int nb = m > 16 ? 4 : m > 8 ? 2 : 1;
-  while (nb > 1 && (size_t)8 * nb * mma_row_pitch(h) > 200 * 1024) nb >>= 1;
-  return nb;
-}
-
-template <int FMT>
-cudaError_t launch_gate_up_mma_fmt(int nb, int grid, size_t smem, cudaStream_t st,
-                                   const Params& p) {
-  switch (nb) {
-    case 1: return launch(gate_up_mma_kernel<FMT, 1>, grid, kThreads, smem, st, p, true);
-    case 2: return launch(gate_up_mma_kernel<FMT, 2>, grid, kThreads, smem, st, p, true);
-    default: return launch(gate_up_mma_kernel<FMT, 4>, grid, kThreads, smem, st, p, true);
-  }
-}
-
-cudaError_t launch_gate_up_mma(int fmt, int nb, int grid, cudaStream_t st, const Params& p) {
-  const size_t smem = (size_t)8 * nb * mma_row_pitch(p.h);
-  switch (fmt) {
-    case MOE_FMT_BF16: return launch_gate_up_mma_fmt<MOE_FMT_BF16>(nb, grid, smem, st, p);
-    case MOE_FMT_FP8_E4M3: return launch_gate_up_mma_fmt<MOE_FMT_FP8_E4M3>(nb, grid, smem, st, p);
-    case MOE_FMT_NVFP4: return launch_gate_up_mma_fmt<MOE_FMT_NVFP4>(nb, grid, smem, st, p);
-    default: return launch_gate_up_mma_fmt<MOE_FMT_MXFP4>(nb, grid, smem, st, p);
-  }
 }
 
 // Rows staged per pass: as many (1, 2 or 4) as fit a 80 KB staging budget, never more than m.
@@ -289,12 +268,9 @@ int sm_count() {
   return cache[dev];
 }
 
-// Debug / test knob, read on every call: MOE_DECODE_PATH=chain forces the three-kernel chain
-// (default: automatic choice).
-int forced_path() {
-  const char* e = std::getenv("MOE_DECODE_PATH");
-  return (e && !std::strcmp(e, "chain")) ? 1 : 0;
-}
+// Launch-path override for tests (moe_debug_set_path): 0 automatic, 1 the multi-kernel chain.
+std::atomic<int> g_forced_path{0};
+int forced_path() { return g_forced_path.load(std::memory_order_relaxed); }
 
 size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
 
@@ -458,6 +434,7 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
                                   const moe_expert_table* shared, const void* shared_gate_w,
                                   void* out, void* workspace, size_t workspace_bytes,
                                   void* stream) {
+  NvtxRange nvtx("moe_decode_forward");
   int rc = check_cfg(cfg, m);
   if (rc) return rc;
   const moe_cfg& c = *cfg;
@@ -533,7 +510,9 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
     FusedPlan fp;
     if (use_fused(c, m, routed, shared, has_shared, &fp)) {
       const cudaError_t e = launch_fused(routed->gate.format, xbf16, m, p, fp, st);
-      return e == cudaSuccess ? MOE_OK : cuda_fail(e);
+      if (e != cudaSuccess) return cuda_fail(e);
+      log_dispatch_once("persistent kernel", routed->gate.format, m, 1);
+      return MOE_OK;
     }
   }
 
@@ -549,16 +528,6 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
   const int fmt_gu = routed->gate.format;
   const bool split_gu = has_shared && shared->gate.format != fmt_gu;
   auto gate_up = [&](int fmt, const Params& q, int grid) {
-    if (mma_gate_up_ok(fmt, xbf16, m, c.hidden)) {
-      // the same launch with 128-row tiles: recount the shared and routed tiles
-      Params qm = q;
-      const bool with_shared = q.n_tiles_s > 0;
-      const bool with_routed = grid > q.n_tiles_s;
-      qm.n_tiles_i = (c.moe_inter + kMmaRowsPerCta - 1) / kMmaRowsPerCta;
-      qm.n_tiles_s = with_shared ? (q.S + kMmaRowsPerCta - 1) / kMmaRowsPerCta : 0;
-      const int gm = qm.n_tiles_s + (with_routed ? q.cap * qm.n_tiles_i : 0);
-      return launch_gate_up_mma(fmt, mma_blocks(c.hidden, m), gm, st, qm);
-    }
     const int rb = rows_per_pass(c.hidden, fmt, m);
     const size_t smem = staging_bytes(c.hidden, fmt, rb);
     return xbf16 ? launch_gate_up<true>(fmt, rb, grid, smem, st, q)
@@ -595,6 +564,8 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
     e = down(fmt_d, p, p.n_tiles_c * (p.cap + p.has_shared), kmax);
   }
   if (e != cudaSuccess) return cuda_fail(e);
+  log_dispatch_once("chain (router, gate/up, down)", routed->gate.format, m,
+                    chain_launches(routed, shared, has_shared));
   return MOE_OK;
 }
 
@@ -613,6 +584,12 @@ extern "C" int moe_decode_launches(const moe_cfg* cfg, int m, const moe_expert_t
   FusedPlan fp;
   *launches = use_fused(*cfg, m, routed, shared, has_shared, &fp)
                   ? 1 : chain_launches(routed, shared, has_shared);
+  return MOE_OK;
+}
+
+extern "C" int moe_debug_set_path(int path) {
+  if (path != 0 && path != 1) return MOE_ERR_BAD_OPTION;
+  g_forced_path.store(path);
   return MOE_OK;
 }
 

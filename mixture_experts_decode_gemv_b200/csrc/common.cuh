@@ -15,8 +15,7 @@ namespace moe {
 // Work-tile geometry shared by the host launcher and the kernels.
 constexpr int kThreads = 256;          // 8 warps per CTA in the expert kernels
 constexpr int kWarps = kThreads / 32;
-constexpr int kLanesPerRow = 8;        // one weight row per 8 lanes, 16 bytes per lane per step
-constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+constexpr int kRowsPerWarp = 4;        // gate/up row pairs a warp reduces, one after another
 constexpr int kRowsPerCta = kWarps * kRowsPerWarp;  // 32 gate/up row pairs per CTA tile
 constexpr int kColsPerCta = 2 * kRowsPerCta;       // 64 down-projection output columns per CTA
 constexpr int kRouterThreads = 128;

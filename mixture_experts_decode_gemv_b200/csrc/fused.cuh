@@ -525,11 +525,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
   }
   __syncthreads();
   MOE_STAMP(9);
-  const unsigned long long tile_mask = s_tile_mask;
-  if (tile_mask && !mbar_wait_bounded(&s_tile_bar, 0, fp.tile_limit)) {
-    atomicExch(p.ctrl + kStatus, (unsigned)MOE_ERR_DEVICE_TIMEOUT);
-    mbar_wait_bounded(&s_tile_bar, 0, fp.tile_limit);  // its copies still target this CTA
+  // Thread 0 waits for the tile's copies and decides for the whole CTA. When the wait runs out
+  // the status records it and every slot is read from global memory instead (same arithmetic);
+  // the copies still target this CTA's shared memory, so the CTA waits for them once more, with
+  // the same bound, before it exits.
+  __shared__ int s_tile_ok;
+  if (tid == 0) {
+    const bool ok = s_tile_mask == 0 || mbar_wait_bounded(&s_tile_bar, 0, fp.tile_limit);
+    if (!ok) atomicExch(p.ctrl + kStatus, (unsigned)MOE_ERR_DEVICE_TIMEOUT);
+    s_tile_ok = ok;
   }
+  __syncthreads();
+  const bool tile_ok = s_tile_ok != 0;
+  const unsigned long long tile_mask = tile_ok ? s_tile_mask : 0ull;
   MOE_STAMP_AFTER(16, (unsigned)tile_mask);
   // units: column pairs of each slot (the routed slots, then the shared expert). A CTA with a
   // down-row tile reads every row through plain loads (tile slots from shared memory, the rest
@@ -605,6 +613,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) moe_fused_kernel(
       reinterpret_cast<float*>(p.out)[o] = acc;
     }
   }
+  if (!tile_ok && tid == 0) mbar_wait_bounded(&s_tile_bar, 0, fp.tile_limit);
   MOE_STAMP(11);
 }
 

@@ -146,28 +146,18 @@ def test_published_shapes_match_oracle(name, m):
     check_out(got if rows is None else got[rows], want)
 
 
-def _mma_chain(cfg) -> bool:
-    """Whether chain calls of this layer may run gate/up on the tensor-core tiles."""
-    kelems = {"bf16": 8, "fp8_e4m3": 16, "nvfp4": 32, "mxfp4": 32}.get(cfg.fmt)
-    return kelems is not None and cfg.x_dtype == "bf16" and cfg.hidden % (4 * kelems) == 0
-
-
 @pytest.mark.parametrize("name", ["ragged_nvfp4_gate", "ragged_q4_shared", "before_ffn_small",
-                                  "mma_fp8_geglu", "mma_mxfp4_bias"])
+                                  "mma_fp8_geglu", "mma_mxfp4_bias", "ragged_bf16",
+                                  "ragged_mxfp4", "tiny_m64"])
 def test_rows_do_not_depend_on_m(name):
-    # Within one launch path a row's bits do not depend on the other rows. Calls of m <= 4 take
-    # the persistent kernel; larger ones the chain, whose gate/up may run on tensor-core tiles
-    # (a different order of the fp32 sums): those rows agree with m = 1 within the tolerance.
+    # A row's bits do not depend on the other rows of the call, nor on m (the grouped decode's
+    # invariant): every launch path reduces each weight row in the same order.
     lay, dev, _ = layer_for(SMALL[name])
     full, _, _ = run(dev, lay.x(64))
     for r in (0, 9, 59):
-        part, _, _ = run(dev, lay.x(5, offset=r))
-        np.testing.assert_array_equal(part, full[r:r + 5])
-        one, _, _ = run(dev, lay.x(1, offset=r))
-        if _mma_chain(dev.cfg):
-            check_out(one[0], full[r].astype(np.float64))
-        else:
-            np.testing.assert_array_equal(one[0], full[r])
+        for n in (1, 2, 5):
+            part, _, _ = run(dev, lay.x(n, offset=r))
+            np.testing.assert_array_equal(part, full[r:r + n])
 
 
 def test_repeated_calls_are_bit_identical_and_workspace_reusable():
@@ -180,15 +170,15 @@ def test_repeated_calls_are_bit_identical_and_workspace_reusable():
         dev.forward(x, out, ws)
         outs.append(out.cpu())
     torch.cuda.synchronize()
-    assert torch.equal(outs[0], outs[2]) and torch.equal(outs[0], outs[4])   # same path, same bits
-    assert torch.equal(outs[1][0], outs[3][0])                               # m = 1 and 4: one kernel
-    # m = 8 takes the chain (tensor-core gate/up): the same rows within the tolerance
-    check_out(outs[1][0].numpy(), outs[0][0].double().numpy())
-    check_out(outs[3].numpy(), outs[0][:4].double().numpy())
+    assert torch.equal(outs[0], outs[2]) and torch.equal(outs[0], outs[4])
+    assert torch.equal(outs[1][0], outs[3][0]) and torch.equal(outs[1][0], outs[0][0])
+    assert torch.equal(outs[3], outs[0][:4])
     assert dev.device_status(ws) == B.MOE_OK
 
 
-def test_bf16_output_is_rounded_fp32_output():
+@pytest.mark.parametrize("m", [1, 3, 8, 40])
+def test_bf16_output_is_rounded_fp32_output(m):
+    # every launch path (the persistent kernel at small m, the multi-kernel path above it)
     cfg = CONFIGS["qwen3_6_35b_a3b"]
     lay, dev, _ = layer_for(cfg)
     dev_b = DeviceLayer.__new__(DeviceLayer)
@@ -196,9 +186,9 @@ def test_bf16_output_is_rounded_fp32_output():
     dev_b.c = type(dev.c).from_buffer_copy(dev.c)
     dev_b.c.out_dtype = B.MOE_FMT_BF16
     dev_b.out_dtype = "bf16"
-    x = dev.x_to_device(lay.x(8))
-    ws = dev.new_workspace(8)
-    o32, o16 = dev.new_out(8), dev_b.new_out(8)
+    x = dev.x_to_device(lay.x(m))
+    ws = dev.new_workspace(m)
+    o32, o16 = dev.new_out(m), dev_b.new_out(m)
     dev.forward(x, o32, ws)
     dev_b.forward(x, o16, ws)
     torch.cuda.synchronize()
@@ -244,23 +234,16 @@ def test_cuda_graph_replay_matches_eager():
 # ---- the two launch paths: one persistent kernel (m <= 4) and the three-kernel chain --------
 
 class _Path:
+    """Force the multi-kernel path ("chain") or restore the automatic choice, for one block."""
+
     def __init__(self, name):
         self.name = name
 
     def __enter__(self):
-        import os
-        self.old = os.environ.get("MOE_DECODE_PATH")
-        if self.name == "chain":
-            os.environ["MOE_DECODE_PATH"] = "chain"
-        else:
-            os.environ.pop("MOE_DECODE_PATH", None)
+        B.moe_debug_set_path(1 if self.name == "chain" else 0)
 
     def __exit__(self, *a):
-        import os
-        if self.old is None:
-            os.environ.pop("MOE_DECODE_PATH", None)
-        else:
-            os.environ["MOE_DECODE_PATH"] = self.old
+        B.moe_debug_set_path(0)
 
 
 PATH_CASES = [(n, m) for n in ("qwen3_30b_a3b", "lfm2_8b_a1b", "qwen3_6_35b_a3b", "llama4_scout",
@@ -320,21 +303,3 @@ def test_grid_barrier_timeout_is_reported_and_the_workspace_recovers():
     torch.cuda.synchronize()
     assert dev.device_status(ws) == B.MOE_OK
     assert torch.equal(out, want)
-
-
-@pytest.mark.parametrize("name", ["max_experts", "mma_fp8_geglu", "mma_mxfp4_bias",
-                                  "mma_bf16_ragged_rows"])
-def test_tensor_core_and_cuda_core_gate_up_agree(name):
-    """The chain's two gate/up implementations on the same call, within the tolerance."""
-    import os
-    lay, dev, _ = layer_for(SMALL[name])
-    x = lay.x(33)
-    try:
-        os.environ["MOE_DECODE_MMA"] = "1"   # tensor-core tiles for every eligible format
-        tc, rt_a, _ = run(dev, x)
-        os.environ["MOE_DECODE_MMA"] = "0"   # CUDA-core tiles
-        cc, rt_b, _ = run(dev, x)
-    finally:
-        os.environ.pop("MOE_DECODE_MMA", None)
-    np.testing.assert_array_equal(rt_a["idx"], rt_b["idx"])
-    check_out(tc, cc.astype(np.float64))

@@ -219,3 +219,93 @@ def test_sqrtsoftplus_bias_changes_the_set_not_the_weights():
     ids, w = ref.route_row(l, cfg, bias)
     assert ids == [1]                                           # 0.4 + bias beats 0.5
     np.testing.assert_allclose(w, [math.sqrt(math.log1p(math.exp(0.4)))], rtol=1e-15)
+
+
+# ---- router GEMV: logits known in closed form ---------------------------------------------------
+
+class _RouterOnly:
+    """A layer source with only the routing inputs (router matrix, bias, shared-gate vector)."""
+
+    def __init__(self, cfg, router_w, expert_bias=None, shared_gate_w=None):
+        self.cfg = cfg
+        self._wr, self._b, self._sg = router_w, expert_bias, shared_gate_w
+
+    def router_w(self):
+        return self._wr
+
+    def expert_bias(self):
+        return self._b
+
+    def shared_gate_w(self):
+        return self._sg
+
+
+def _bf16_bits(v):
+    """bfloat16 storage of values that bf16 holds exactly (small integers, powers of two)."""
+    b = np.asarray(v, dtype=np.float32).view(np.uint32)
+    assert np.all(b & 0xFFFF == 0), "value not exact in bf16"
+    return (b >> 16).astype(np.uint16)
+
+
+def test_router_logits_of_scaled_basis_rows():
+    # E = 5 router rows over h = 12 inputs, row e = c_e * (unit vector at position p_e), so
+    # logit[r, e] = c_e * x[r, p_e] exactly; m = 3 rows (m, E and h all differ, so a transposed
+    # operand or a swapped index cannot produce the right [m, E] array).
+    E, h, m = 5, 12, 3
+    pos = [3, 0, 11, 7, 5]
+    c = [2.0, -1.0, 0.5, 3.0, -4.0]
+    wr = np.zeros((E, h), np.float32)
+    for e in range(E):
+        wr[e, pos[e]] = c[e]
+    x = np.arange(m * h, dtype=np.float32).reshape(m, h) - 17.0   # integers -17 .. 18
+    want = np.array([[c[e] * x[r, pos[e]] for e in range(E)] for r in range(m)])
+    cfg = cfg_of(hidden=h, num_experts=E, top_k=2, x_dtype="f32", fmt="f32")
+    rt = ref.route(ref.OracleLayer(_RouterOnly(cfg, wr)), x)
+    assert rt["logits"].shape == (m, E)
+    np.testing.assert_array_equal(rt["logits"], want)
+    for r in range(m):
+        order = sorted(range(E), key=lambda e: (-want[r, e], e))[:2]
+        assert list(rt["idx"][r]) == order
+        p = [math.exp(want[r, e]) for e in order]                 # renormalised softmax
+        np.testing.assert_allclose(rt["w"][r], [v / sum(p) for v in p], rtol=1e-14)
+
+
+def test_router_logits_of_integer_rows_in_bf16():
+    # bf16 router rows and activations holding small integers: every logit is an integer that
+    # plain Python integer arithmetic gives exactly.
+    rng = np.random.default_rng(7)
+    E, h, m = 7, 16, 4
+    wr = rng.integers(-3, 4, size=(E, h))
+    x = rng.integers(-5, 6, size=(m, h))
+    want = [[sum(int(wr[e, j]) * int(x[r, j]) for j in range(h)) for e in range(E)]
+            for r in range(m)]
+    cfg = cfg_of(hidden=h, num_experts=E, top_k=3, x_dtype="bf16", fmt="bf16")
+    rt = ref.route(ref.OracleLayer(_RouterOnly(cfg, _bf16_bits(wr))), _bf16_bits(x))
+    np.testing.assert_array_equal(rt["logits"], np.array(want, dtype=np.float64))
+    for r in range(m):
+        assert list(rt["idx"][r]) == sorted(range(E), key=lambda e: (-want[r][e], e))[:3]
+
+
+def test_router_sigmoid_bias_and_shared_gate_from_known_logits():
+    # Logits set by basis rows; the bias changes the winner while the weights stay the unbiased
+    # sigmoid scores; the shared gate is sigmoid of x at the gate vector's one non-zero position.
+    E, h = 4, 6
+    wr = np.zeros((E, h), np.float32)
+    for e, (p, c) in enumerate([(1, 1.0), (4, 1.0), (0, 2.0), (5, -1.0)]):
+        wr[e, p] = c
+    x = np.array([[0.5, 1.0, -2.0, 0.0, 0.75, 0.25]], np.float32)
+    logits = [1.0, 0.75, 1.0, -0.25]                 # x[1], x[4], 2 x[0], -x[5]
+    bias = np.array([0.0, 0.5, -0.4, 0.0], np.float32)
+    sg = np.zeros(h, np.float32)
+    sg[2] = 0.5                                     # w_sg . x = -1
+    cfg = cfg_of(hidden=h, num_experts=E, top_k=2, x_dtype="f32", fmt="f32", routing="sigmoid",
+                 has_expert_bias=True, norm_topk_prob=False, routed_scaling_factor=2.0,
+                 shared_inter=4, shared_kind="sigmoid_gate")
+    rt = ref.route(ref.OracleLayer(_RouterOnly(cfg, wr, bias, sg)), x)
+    np.testing.assert_array_equal(rt["logits"][0], logits)
+    sig = [1.0 / (1.0 + math.exp(-v)) for v in logits]
+    keys = [sig[e] + float(bias[e]) for e in range(E)]   # 0.731, 1.179, 0.331, 0.438
+    assert list(rt["idx"][0]) == [1, 0]
+    assert sorted(range(E), key=lambda e: -keys[e])[:2] == [1, 0]
+    np.testing.assert_allclose(rt["w"][0], [2.0 * sig[1], 2.0 * sig[0]], rtol=1e-14)
+    np.testing.assert_allclose(rt["gamma"], [1.0 / (1.0 + math.e)], rtol=1e-14)
