@@ -53,8 +53,17 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     monkeypatch.setenv("RANK", "1")
     args = argparse.Namespace(m=1, steps=1, warmup=0)
-    bench.run_reference(args, CONFIGS["tiny"])
+    bench.run_reference(args, CONFIGS["tiny"], 1)
     assert capsys.readouterr().out == ""
+
+
+def test_both_arms_print_the_same_config():
+    import bench
+    from mixture_experts_decode_gemv_b200.synthetic import CONFIGS
+    c = CONFIGS["llama4_scout"]
+    assert bench.config_dict(c, 64, 1) == bench.config_dict(c, 64, 1)
+    assert set(bench.config_dict(c, 64, 1)) == {"workload", "m", "weights", "l2_policy",
+                                                 "parallelism"}
 
 
 def test_single_rank_helpers_need_no_process_group():
