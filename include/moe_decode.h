@@ -200,6 +200,15 @@ int moe_debug_barrier_test(int extra_arrivals, long long spin_limit_cycles);
  * decode pages have no counterpart. */
 int moe_debug_set_path(int path);
 
+/* Test aid: how the tensor-core path shares out its work in every later forward call in this
+ * process. mode 0 is the automatic choice; 1 gives every job (32 weight rows of one expert
+ * projection) to one warp; 2 splits jobs into 256-element pieces of the reduction wherever the
+ * workspace holds their partial values. The results are the same bits in every mode (the pieces'
+ * values are summed in one fixed order); tests use this to check that. Process-wide; do not call
+ * it while other threads run forward calls. Returns MOE_ERR_BAD_OPTION for other values. The
+ * decode pages have no counterpart. */
+int moe_debug_set_split(int mode);
+
 /* Copy the routing and grouping of the last forward call that used `workspace` to host arrays
  * (synchronises `stream`). Any output pointer may be NULL to skip it. Sizes: idx, weights,
  * sorted_pairs, token_to_perm: m*top_k; expert_offsets: num_experts+1; active: min(m*top_k, E);

@@ -54,7 +54,7 @@ EXPORTS = (
     "moe_quantize_nvfp4", "moe_dequantize", "moe_status_string", "moe_last_cuda_error",
     "moe_version", "moe_decode_forward_no_alloc", "moe_decode_launches",
     "moe_debug_barrier_test", "moe_quantize_mxfp4", "moe_quantize_fp8_e4m3",
-    "moe_debug_set_path",
+    "moe_debug_set_path", "moe_debug_set_split",
 )
 
 MOE_NO_ALLOC_SCRATCH_BYTES = 16 << 20
@@ -122,6 +122,7 @@ def _load() -> ctypes.CDLL:
                                 P(ctypes.c_int32)],
         "moe_debug_barrier_test": [i32, i64],
         "moe_debug_set_path": [i32],
+        "moe_debug_set_split": [i32],
         "moe_status_string": [i32],
         "moe_last_cuda_error": [],
         "moe_version": [],
@@ -218,6 +219,11 @@ def moe_debug_barrier_test(extra_arrivals: int, spin_limit_cycles: int) -> None:
 def moe_debug_set_path(path: int) -> None:
     """Test aid: 0 automatic launch path, 1 the multi-kernel path at every m (process-wide)."""
     _check(lib.moe_debug_set_path(path), "moe_debug_set_path")
+
+
+def moe_debug_set_split(mode: int) -> None:
+    """Test aid: 0 automatic work split, 1 whole jobs per warp, 2 jobs split by chunk."""
+    _check(lib.moe_debug_set_split(mode), "moe_debug_set_split")
 
 
 def moe_decode_read_routing(cfg: moe_cfg, m: int, workspace, workspace_bytes: int, stream=None):

@@ -16,6 +16,7 @@
 #include "experts.cuh"
 #include "fused.cuh"
 #include "router.cuh"
+#include "tc.cuh"
 
 using namespace moe;
 
@@ -123,9 +124,94 @@ int check_table(const moe_expert_table* t, int inter, int h, int E, MatDev* g, M
 
 int n_tiles_c_of(int h) { return (h + kColsPerCta - 1) / kColsPerCta; }
 
-WsLayout layout_of(const moe_cfg* c, int m) {
+// ---- tensor-core path: work shape and workspace regions ----------------------------------------
+
+// Split jobs keep their chunk values in the workspace: 32 floats per (activation column, job
+// tile, chunk). A phase may split its jobs when that storage stays within this size.
+constexpr size_t kSlotCapBytes = 24u << 20;
+
+// Everything the tensor-core regions and work split depend on, from (cfg, m) alone.
+struct TcShape {
+  int ntg, ncg_max, tiles_i, tiles_s, tiles_h, nch_h, nch_i, nch_s;
+  int j_gu_max, j_dn_max;
+  size_t gu_bytes, dn_bytes;           // chunk-value storage of the two phases
+  bool gu_slots, dn_slots;             // within the cap: the phase may split its jobs
+};
+
+TcShape tc_shape(const moe_cfg& c, int m) {
+  TcShape t;
+  const bool has_shared = c.shared_kind != MOE_SHARED_NONE;
+  const int S = has_shared ? c.shared_inter : 0;
+  t.ntg = m <= 8 ? 1 : m <= 16 ? 2 : 4;   // n-tiles of 8 activation columns per pass (bf16;
+                                          // the other formats take at most 2)
+  t.ncg_max = tc::ceil_div(m, 8 * (t.ntg < 2 ? t.ntg : 2));  // column groups at the smallest width
+  t.tiles_i = tc::ceil_div(c.moe_inter, 16);
+  t.tiles_s = S ? tc::ceil_div(S, 16) : 0;
+  t.tiles_h = tc::ceil_div(c.hidden, 32);
+  t.nch_h = tc::n_chunks(c.hidden);
+  t.nch_i = tc::n_chunks(c.moe_inter);
+  t.nch_s = S ? tc::n_chunks(S) : 1;
+  const int te = m * c.top_k;
+  const int cap = te < c.num_experts ? te : c.num_experts;
+  t.j_gu_max = cap * t.tiles_i + t.tiles_s;
+  t.j_dn_max = (cap + (has_shared ? 1 : 0)) * t.tiles_h;
+  t.gu_bytes = ((size_t)te * t.tiles_i + (size_t)m * t.tiles_s) * t.nch_h * 32 * 4;
+  t.dn_bytes = ((size_t)te * t.tiles_h * t.nch_i + (has_shared ? (size_t)m * t.tiles_h * t.nch_s : 0)) *
+               32 * 4;
+  t.gu_slots = t.gu_bytes <= kSlotCapBytes;
+  t.dn_slots = t.dn_bytes <= kSlotCapBytes;
+  return t;
+}
+
+struct TcLayout {
+  size_t xb, act, sh_act, slot_beg, slot_n, gu_slots, dn_slots, tk, stamps, end;
+  int tk_words;
+};
+
+TcLayout tc_layout(const moe_cfg& c, int m, size_t off) {
+  const TcShape t = tc_shape(c, m);
+  const bool has_shared = c.shared_kind != MOE_SHARED_NONE;
+  const int S = has_shared ? c.shared_inter : 0;
+  const size_t te = (size_t)m * c.top_k;
+  const size_t cap = te < (size_t)c.num_experts ? te : (size_t)c.num_experts;
+  TcLayout L;
+  auto take = [&](size_t bytes) { size_t at = off; off = align256(off + bytes); return at; };
+  L.xb = take((size_t)m * c.hidden * 2);
+  L.act = take(te * c.moe_inter * 4);                   // hi and lo halves
+  L.sh_act = take((size_t)m * (S > 0 ? S : 1) * 4);
+  L.slot_beg = take(cap * 4);
+  L.slot_n = take(cap * 4);
+  // slot storage: the most any call with at most m rows uses, so that the workspace size only
+  // grows with m (a workspace sized for the largest m serves every smaller one)
+  size_t gu_bytes = 0, dn_bytes = 0;
+  for (int mm = 1; mm <= m; ++mm) {
+    const TcShape u = tc_shape(c, mm);
+    if (u.gu_slots && u.gu_bytes > gu_bytes) gu_bytes = u.gu_bytes;
+    if (u.dn_slots && u.dn_bytes > dn_bytes) dn_bytes = u.dn_bytes;
+  }
+  L.gu_slots = take(gu_bytes);
+  L.dn_slots = take(dn_bytes);
+  L.tk_words = (t.j_gu_max + t.j_dn_max) * t.ncg_max + t.tiles_h;
+  L.tk = take((size_t)L.tk_words * 4);
+#ifdef MOE_PHASE_TIMERS
+  L.stamps = take((size_t)1024 * 16 * 8);  // [CTA][16] uint64, last region of the workspace
+#else
+  L.stamps = 0;
+#endif
+  L.end = off;
+  return L;
+}
+
+WsLayout base_layout_of(const moe_cfg* c, int m) {
   return make_layout(m, c->hidden, c->num_experts, c->top_k, c->moe_inter, c->shared_inter,
                      n_tiles_c_of(c->hidden));
+}
+
+// The whole workspace: the regions every path uses, then the tensor-core path's.
+WsLayout layout_of(const moe_cfg* c, int m) {
+  WsLayout L = base_layout_of(c, m);
+  L.total = tc_layout(*c, m, L.total).end;
+  return L;
 }
 
 // NVTX range around a library call (visible in Nsight timelines; a few ns when no tool listens).
@@ -271,6 +357,9 @@ int sm_count() {
 // Launch-path override for tests (moe_debug_set_path): 0 automatic, 1 the multi-kernel chain.
 std::atomic<int> g_forced_path{0};
 int forced_path() { return g_forced_path.load(std::memory_order_relaxed); }
+// Work-split override for tests (moe_debug_set_split): 0 automatic, 1 whole jobs per warp,
+// 2 jobs split by chunk wherever the workspace holds their chunk values.
+std::atomic<int> g_forced_split{0};
 
 size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
 
@@ -391,6 +480,113 @@ cudaError_t launch_fused(int fmt, bool xbf16, int m, const Params& p, const Fuse
   }
 }
 
+// The tensor-core path takes a call when one format in {bf16, FP8, NVFP4, MXFP4, Q4} serves
+// every projection, the activations are bf16, and (fp16 operand formats) hidden is a multiple of
+// 16 (the activations are converted in 16-element blocks).
+bool tc_eligible(const moe_cfg& c, const moe_expert_table* routed, const moe_expert_table* shared,
+                 bool has_shared) {
+  const int fmt = routed->gate.format;
+  if (fmt == MOE_FMT_F32 || c.x_dtype != MOE_FMT_BF16) return false;
+  if (routed->down.format != fmt) return false;
+  if (has_shared && (shared->gate.format != fmt || shared->down.format != fmt)) return false;
+  if (fmt != MOE_FMT_BF16 && c.hidden % 16) return false;
+  // scale and bias slabs are read as aligned 4-byte words: their bases must be 4-byte aligned
+  auto words_ok = [](const moe_matrix& M) {
+    return (!M.scales || aligned(M.scales, 4)) && (!M.biases || aligned(M.biases, 4));
+  };
+  if (!words_ok(routed->gate) || !words_ok(routed->up) || !words_ok(routed->down)) return false;
+  if (has_shared && (!words_ok(shared->gate) || !words_ok(shared->up) || !words_ok(shared->down)))
+    return false;
+  return true;
+}
+
+template <typename K>
+cudaError_t launch_tc(K kernel, int grid, int block, cudaStream_t st, bool cooperative,
+                      const Params& p, const tc::TcExtra& tx, const tc::TcPlan* pl,
+                      const int* slot_beg, const int* slot_n) {
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               tc::kRingWarpsBytes);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = tc::kRingWarpsBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (cooperative) {
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  if constexpr (std::is_invocable_v<K, Params, tc::TcExtra, tc::TcPlan>) {
+    return cudaLaunchKernelEx(&cfg, kernel, p, tx, *pl);
+  } else {
+    return cudaLaunchKernelEx(&cfg, kernel, p, tx, slot_beg, slot_n);
+  }
+}
+
+template <int FMT, int NTG>
+cudaError_t tc_run(bool chain, int sms, cudaStream_t st, const Params& p, const tc::TcExtra& tx,
+                   const tc::TcPlan& pl, int* slot_beg, int* slot_n) {
+  if (!chain) {
+    auto kernel = tc::tc_fused_kernel<FMT, NTG>;
+    int per_sm = 0;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         tc::kRingWarpsBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, tc::kThreads,
+                                                      tc::kRingWarpsBytes);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+    return launch_tc(kernel, sms, tc::kThreads, st, true, p, tx, &pl, nullptr, nullptr);
+  }
+  const int router_grid = p.E + (p.shared_kind == MOE_SHARED_SIGMOID_GATE ? 1 : 0);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(router_grid);
+  cfg.blockDim = dim3(kRouterThreads);
+  cfg.stream = st;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tc::tc_router_kernel<FMT>, p, tx, slot_beg, slot_n);
+  if (e != cudaSuccess) return e;
+  e = launch_tc(tc::tc_gate_up_kernel<FMT, NTG>, sms, tc::kThreads, st, false, p, tx, nullptr,
+                slot_beg, slot_n);
+  if (e != cudaSuccess) return e;
+  return launch_tc(tc::tc_down_kernel<FMT, NTG>, sms, tc::kThreads, st, false, p, tx, nullptr,
+                   slot_beg, slot_n);
+}
+
+template <int FMT>
+cudaError_t tc_run_ntg(int ntg, bool chain, int sms, cudaStream_t st, const Params& p,
+                       const tc::TcExtra& tx, const tc::TcPlan& pl, int* sb, int* sn) {
+  if constexpr (FMT == MOE_FMT_BF16) {
+    if (ntg == 4) return tc_run<FMT, 4>(chain, sms, st, p, tx, pl, sb, sn);
+  }
+  return ntg == 1 ? tc_run<FMT, 1>(chain, sms, st, p, tx, pl, sb, sn)
+                  : tc_run<FMT, 2>(chain, sms, st, p, tx, pl, sb, sn);
+}
+
+cudaError_t tc_launch(int fmt, int ntg, bool chain, int sms, cudaStream_t st, const Params& p,
+                      const tc::TcExtra& tx, const tc::TcPlan& pl, int* sb, int* sn) {
+  switch (fmt) {
+    case MOE_FMT_BF16: return tc_run_ntg<MOE_FMT_BF16>(ntg, chain, sms, st, p, tx, pl, sb, sn);
+    case MOE_FMT_FP8_E4M3:
+      return tc_run_ntg<MOE_FMT_FP8_E4M3>(ntg, chain, sms, st, p, tx, pl, sb, sn);
+    case MOE_FMT_NVFP4: return tc_run_ntg<MOE_FMT_NVFP4>(ntg, chain, sms, st, p, tx, pl, sb, sn);
+    case MOE_FMT_MXFP4: return tc_run_ntg<MOE_FMT_MXFP4>(ntg, chain, sms, st, p, tx, pl, sb, sn);
+    default:
+      return tc_run_ntg<MOE_FMT_Q4_AFFINE_G64>(ntg, chain, sms, st, p, tx, pl, sb, sn);
+  }
+}
+
 }  // namespace
 
 extern "C" int moe_workspace_bytes(const moe_cfg* cfg, int m, size_t* out_bytes) {
@@ -506,6 +702,56 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
   cudaStream_t st = (cudaStream_t)stream;
   const bool xbf16 = c.x_dtype == MOE_FMT_BF16;
 
+  if (tc_eligible(c, routed, shared, has_shared)) {
+    const TcShape ts = tc_shape(c, m);
+    const TcLayout tl = tc_layout(c, m, base_layout_of(&c, m).total);
+    const int sms = sm_count();
+    if (sms <= 0) return MOE_ERR_UNSUPPORTED_DEVICE;
+    tc::TcExtra tx;
+    std::memset(&tx, 0, sizeof(tx));
+    tx.W = sms * tc::kWarps;
+    const int split = g_forced_split.load(std::memory_order_relaxed);
+    tx.gu_piece = ts.gu_slots && (split == 2 || (split == 0 && ts.j_gu_max < 4 * tx.W));
+    // down jobs are split only when their rows come from HBM: when every active expert's down
+    // rows fit the L2 prefetch (asked for during gate/up), whole jobs read them from L2 with
+    // fewer serial round trips
+    const size_t down_max = ((size_t)p.cap * packed_row_bytes(routed->down.format, c.moe_inter) +
+                             (has_shared ? packed_row_bytes(routed->down.format, p.S) : 0)) *
+                            (size_t)c.hidden;
+    const long long l2_cap = 48LL << 20;
+    tx.dn_piece = ts.dn_slots && (split == 2 || (split == 0 && ts.j_dn_max < 4 * tx.W &&
+                                                 down_max > (size_t)l2_cap));
+    tx.tiles_i = ts.tiles_i;
+    tx.tiles_s = ts.tiles_s;
+    tx.tiles_h = ts.tiles_h;
+    tx.nch_h = ts.nch_h;
+    tx.nch_i = ts.nch_i;
+    tx.nch_s = ts.nch_s;
+    tx.xb = ws + tl.xb;
+    tx.act = ws + tl.act;
+    tx.sh_act = ws + tl.sh_act;
+    tx.gu_slots = (float*)(ws + tl.gu_slots);
+    tx.dn_slots = (float*)(ws + tl.dn_slots);
+    tx.tk_gu = (unsigned*)(ws + tl.tk);
+    tx.tk_dn = tx.tk_gu + (size_t)ts.j_gu_max * ts.ncg_max;
+    tx.tk_col = tx.tk_dn + (size_t)ts.j_dn_max * ts.ncg_max;
+    tx.tk_words = tl.tk_words;
+    tx.stamps = tl.stamps ? (unsigned long long*)(ws + tl.stamps) : nullptr;
+    tc::TcPlan pl;
+    pl.spin_limit = g_test_spin_limit.load() > 0 ? g_test_spin_limit.load() : kSpinLimit;
+    pl.bar_extra = (unsigned)g_test_bar_extra.load();
+    pl.l2_prefetch_cap = l2_cap;
+    const bool chain = forced_path() == 1;
+    const int ntg = routed->gate.format == MOE_FMT_BF16 ? ts.ntg : (ts.ntg < 2 ? ts.ntg : 2);
+    const cudaError_t e = tc_launch(routed->gate.format, ntg, chain, sms, st, p, tx, pl,
+                                    (int*)(ws + tl.slot_beg), (int*)(ws + tl.slot_n));
+    if (e != cudaSuccess) return cuda_fail(e);
+    log_dispatch_once(chain ? "chain (tensor-core router, gate/up, down)"
+                            : "persistent tensor-core kernel",
+                      routed->gate.format, m, chain ? 3 : 1);
+    return MOE_OK;
+  }
+
   {
     FusedPlan fp;
     if (use_fused(c, m, routed, shared, has_shared, &fp)) {
@@ -582,14 +828,24 @@ extern "C" int moe_decode_launches(const moe_cfg* cfg, int m, const moe_expert_t
     return rc;
   if ((rc = check_device())) return rc;
   FusedPlan fp;
-  *launches = use_fused(*cfg, m, routed, shared, has_shared, &fp)
-                  ? 1 : chain_launches(routed, shared, has_shared);
+  if (tc_eligible(*cfg, routed, shared, has_shared)) {
+    *launches = forced_path() == 1 ? 3 : 1;
+  } else {
+    *launches = use_fused(*cfg, m, routed, shared, has_shared, &fp)
+                    ? 1 : chain_launches(routed, shared, has_shared);
+  }
   return MOE_OK;
 }
 
 extern "C" int moe_debug_set_path(int path) {
   if (path != 0 && path != 1) return MOE_ERR_BAD_OPTION;
   g_forced_path.store(path);
+  return MOE_OK;
+}
+
+extern "C" int moe_debug_set_split(int mode) {
+  if (mode < 0 || mode > 2) return MOE_ERR_BAD_OPTION;
+  g_forced_split.store(mode);
   return MOE_OK;
 }
 

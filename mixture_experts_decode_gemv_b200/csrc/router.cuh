@@ -66,6 +66,45 @@ __device__ __forceinline__ float router_dot_warp(const uint8_t* row, int nch, XC
   return warp_sum(acc);
 }
 
+// The same dot product (same chunk order per lane, same fma order, same butterfly sum) with the
+// activation row in global memory: the weight and activation loads of up to 8 chunks per lane
+// are issued together before any is used, so a chunk's activations cost no extra round trip.
+template <bool XBF16>
+__device__ __forceinline__ float router_dot_gx(const uint8_t* row, const uint8_t* xr, int nch) {
+  const int lane = threadIdx.x & 31;
+  float acc = 0.f;
+  for (int c0 = lane; c0 < nch; c0 += 32 * 8) {
+    uint4 w[8], x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (c0 + 32 * u < nch) {
+        w[u] = ldg_stream(row + (size_t)(c0 + 32 * u) * 16);
+        x[u] = __ldg(reinterpret_cast<const uint4*>(xr) + c0 + 32 * u);
+      }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (c0 + 32 * u < nch) {
+        if constexpr (XBF16) {
+          acc = fmaf(bf16lo(w[u].x), bf16lo(x[u].x), acc);
+          acc = fmaf(bf16hi(w[u].x), bf16hi(x[u].x), acc);
+          acc = fmaf(bf16lo(w[u].y), bf16lo(x[u].y), acc);
+          acc = fmaf(bf16hi(w[u].y), bf16hi(x[u].y), acc);
+          acc = fmaf(bf16lo(w[u].z), bf16lo(x[u].z), acc);
+          acc = fmaf(bf16hi(w[u].z), bf16hi(x[u].z), acc);
+          acc = fmaf(bf16lo(w[u].w), bf16lo(x[u].w), acc);
+          acc = fmaf(bf16hi(w[u].w), bf16hi(x[u].w), acc);
+        } else {
+          acc = fmaf(__uint_as_float(w[u].x), __uint_as_float(x[u].x), acc);
+          acc = fmaf(__uint_as_float(w[u].y), __uint_as_float(x[u].y), acc);
+          acc = fmaf(__uint_as_float(w[u].z), __uint_as_float(x[u].z), acc);
+          acc = fmaf(__uint_as_float(w[u].w), __uint_as_float(x[u].w), acc);
+        }
+      }
+    }
+  }
+  return warp_sum(acc);
+}
+
 // Order-preserving map of a float key to uint32 (NaN ranks as -infinity).
 __device__ __forceinline__ uint32_t key_bits(float v) {
   if (v != v) v = -INFINITY;
@@ -347,16 +386,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_group_kernel(
   // one warp per activation row; the router row comes from L2 after the first warp's pass
   for (int r = warp; r < p.m; r += kRouterThreads / 32) {
     const uint8_t* xr = xb + (size_t)r * row_bytes;
-    const float acc = router_dot_warp<XBF16>(wrow, nch, [&](int c, float* xv) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr) + c);
-      if constexpr (XBF16) {
-        xv[0] = bf16lo(v.x); xv[1] = bf16hi(v.x); xv[2] = bf16lo(v.y); xv[3] = bf16hi(v.y);
-        xv[4] = bf16lo(v.z); xv[5] = bf16hi(v.z); xv[6] = bf16lo(v.w); xv[7] = bf16hi(v.w);
-      } else {
-        xv[0] = __uint_as_float(v.x); xv[1] = __uint_as_float(v.y);
-        xv[2] = __uint_as_float(v.z); xv[3] = __uint_as_float(v.w);
-      }
-    });
+    const float acc = router_dot_gx<XBF16>(wrow, xr, nch);
     if (lane == 0) p.logits[(size_t)r * (p.E + 1) + erow] = acc;
   }
   __syncthreads();

@@ -175,6 +175,9 @@ def test_barrier_test_hook_validates_its_arguments():
     assert B.lib.moe_debug_set_path(2) == B.MOE_ERR_BAD_OPTION
     assert B.lib.moe_debug_set_path(-1) == B.MOE_ERR_BAD_OPTION
     assert B.lib.moe_debug_set_path(0) == B.MOE_OK
+    assert B.lib.moe_debug_set_split(3) == B.MOE_ERR_BAD_OPTION
+    assert B.lib.moe_debug_set_split(-1) == B.MOE_ERR_BAD_OPTION
+    assert B.lib.moe_debug_set_split(0) == B.MOE_OK
 
 
 # ---- pack / quantise helpers ---------------------------------------------------------------

@@ -246,9 +246,11 @@ class _Path:
         B.moe_debug_set_path(0)
 
 
-PATH_CASES = [(n, m) for n in ("qwen3_30b_a3b", "lfm2_8b_a1b", "qwen3_6_35b_a3b", "llama4_scout",
-                                "qwen3_30b_a3b_mxfp4", "qwen3_30b_a3b_fp8")
-              for m in (1, 2, 3, 4)] + [(n, m) for n in SMALL for m in (1, 4)]
+PATH_CASES = ([(n, m) for n in ("qwen3_30b_a3b", "lfm2_8b_a1b", "qwen3_6_35b_a3b", "llama4_scout",
+                                 "qwen3_30b_a3b_mxfp4", "qwen3_30b_a3b_fp8")
+               for m in (1, 2, 3, 4)]
+              + [(n, m) for n in SMALL for m in (1, 4, 9, 40)]
+              + [("lfm2_8b_a1b", 16), ("qwen3_6_35b_a3b", 16), ("qwen3_30b_a3b", 8)])
 
 
 @pytest.mark.parametrize("name,m", PATH_CASES)
@@ -271,11 +273,54 @@ def test_persistent_kernel_and_chain_agree_bitwise(name, m):
 
 
 def test_launch_count_follows_the_dispatch_rule():
+    # tensor-core formats: one persistent launch at every m (three when the chain is forced);
+    # f32 weights: the persistent CUDA-core kernel up to m = 4, the chain above
     lay, dev, _ = layer_for(CONFIGS["qwen3_30b_a3b"])
-    assert [dev.launches(m) for m in (1, 2, 3, 4)] == [1, 1, 1, 1]
-    assert [dev.launches(m) for m in (5, 8, 64)] == [3, 3, 3]
+    assert [dev.launches(m) for m in (1, 2, 3, 4, 5, 8, 64)] == [1] * 7
     with _Path("chain"):
-        assert dev.launches(1) == 3
+        assert dev.launches(1) == 3 and dev.launches(64) == 3
+    lay, dev, _ = layer_for(SMALL["tiny_m64"])
+    assert [dev.launches(m) for m in (1, 4, 5, 64)] == [1, 1, 3, 3]
+
+
+class _Split:
+    """Force a work split of the tensor-core path for one block (0 automatic, 1 whole jobs,
+    2 jobs split by chunk)."""
+
+    def __init__(self, mode):
+        self.mode = mode
+
+    def __enter__(self):
+        B.moe_debug_set_split(self.mode)
+
+    def __exit__(self, *a):
+        B.moe_debug_set_split(0)
+
+
+SPLIT_CASES = [("ragged_bf16", 17), ("ragged_q4_shared", 3), ("ragged_nvfp4_gate", 40),
+               ("ragged_mxfp4", 9), ("ragged_fp8_geglu", 64), ("max_experts", 64),
+               ("k_equals_E", 40), ("qwen3_30b_a3b", 1), ("lfm2_8b_a1b", 4),
+               ("qwen3_6_35b_a3b", 16)]
+
+
+@pytest.mark.parametrize("name,m", SPLIT_CASES)
+def test_work_split_does_not_change_the_bits(name, m):
+    # whole jobs per warp and jobs split into 256-element pieces give identical outputs, on
+    # both launch paths
+    cfg = SMALL.get(name) or CONFIGS[name]
+    lay, dev, olay = layer_for(cfg)
+    x = lay.x(m, offset=1 if m < 64 else 0)
+    outs = []
+    for path in ("auto", "chain"):
+        for mode in (1, 2, 0):
+            with _Path(path), _Split(mode):
+                got, _, st = run(dev, x)
+            assert st == B.MOE_OK
+            outs.append(got)
+    for o in outs[1:]:
+        np.testing.assert_array_equal(o, outs[0])
+    want, _ = ref.moe_forward(olay, x)
+    check_out(outs[0], want)
 
 
 def test_grid_barrier_timeout_is_reported_and_the_workspace_recovers():
