@@ -138,7 +138,9 @@ struct TcShape {
   bool gu_slots, dn_slots;             // within the cap: the phase may split its jobs
 };
 
-TcShape tc_shape(const moe_cfg& c, int m) {
+// fmt: the format whose chunk size counts the chunks; the workspace is sized with bf16's, the
+// smallest chunk (the most chunks).
+TcShape tc_shape(const moe_cfg& c, int m, int fmt = MOE_FMT_BF16) {
   TcShape t;
   const bool has_shared = c.shared_kind != MOE_SHARED_NONE;
   const int S = has_shared ? c.shared_inter : 0;
@@ -148,9 +150,9 @@ TcShape tc_shape(const moe_cfg& c, int m) {
   t.tiles_i = tc::ceil_div(c.moe_inter, 16);
   t.tiles_s = S ? tc::ceil_div(S, 16) : 0;
   t.tiles_h = tc::ceil_div(c.hidden, 32);
-  t.nch_h = tc::n_chunks(c.hidden);
-  t.nch_i = tc::n_chunks(c.moe_inter);
-  t.nch_s = S ? tc::n_chunks(S) : 1;
+  t.nch_h = tc::n_chunks(c.hidden, fmt);
+  t.nch_i = tc::n_chunks(c.moe_inter, fmt);
+  t.nch_s = S ? tc::n_chunks(S, fmt) : 1;
   const int te = m * c.top_k;
   const int cap = te < c.num_experts ? te : c.num_experts;
   t.j_gu_max = cap * t.tiles_i + t.tiles_s;
@@ -508,13 +510,13 @@ cudaError_t launch_tc(K kernel, int grid, int block, cudaStream_t st, bool coope
   {
     std::lock_guard<std::mutex> lock(mu);
     const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               tc::kRingWarpsBytes);
+                                               tc::kRingCtaBytes);
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(block);
-  cfg.dynamicSmemBytes = tc::kRingWarpsBytes;
+  cfg.dynamicSmemBytes = tc::kRingCtaBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   int na = 0;
@@ -538,17 +540,17 @@ cudaError_t launch_tc(K kernel, int grid, int block, cudaStream_t st, bool coope
 template <int FMT, int NTG>
 cudaError_t tc_run(bool chain, int sms, cudaStream_t st, const Params& p, const tc::TcExtra& tx,
                    const tc::TcPlan& pl, int* slot_beg, int* slot_n) {
+  constexpr int kThr = 32 * tc::tc_warps<FMT, NTG>();
   if (!chain) {
     auto kernel = tc::tc_fused_kernel<FMT, NTG>;
     int per_sm = 0;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         tc::kRingWarpsBytes);
+                                         tc::kRingCtaBytes);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, tc::kThreads,
-                                                      tc::kRingWarpsBytes);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThr, tc::kRingCtaBytes);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
-    return launch_tc(kernel, sms, tc::kThreads, st, true, p, tx, &pl, nullptr, nullptr);
+    return launch_tc(kernel, sms, kThr, st, true, p, tx, &pl, nullptr, nullptr);
   }
   const int router_grid = p.E + (p.shared_kind == MOE_SHARED_SIGMOID_GATE ? 1 : 0);
   cudaLaunchConfig_t cfg = {};
@@ -557,10 +559,10 @@ cudaError_t tc_run(bool chain, int sms, cudaStream_t st, const Params& p, const 
   cfg.stream = st;
   cudaError_t e = cudaLaunchKernelEx(&cfg, tc::tc_router_kernel<FMT>, p, tx, slot_beg, slot_n);
   if (e != cudaSuccess) return e;
-  e = launch_tc(tc::tc_gate_up_kernel<FMT, NTG>, sms, tc::kThreads, st, false, p, tx, nullptr,
+  e = launch_tc(tc::tc_gate_up_kernel<FMT, NTG>, sms, kThr, st, false, p, tx, nullptr,
                 slot_beg, slot_n);
   if (e != cudaSuccess) return e;
-  return launch_tc(tc::tc_down_kernel<FMT, NTG>, sms, tc::kThreads, st, false, p, tx, nullptr,
+  return launch_tc(tc::tc_down_kernel<FMT, NTG>, sms, kThr, st, false, p, tx, nullptr,
                    slot_beg, slot_n);
 }
 
@@ -703,13 +705,13 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
   const bool xbf16 = c.x_dtype == MOE_FMT_BF16;
 
   if (tc_eligible(c, routed, shared, has_shared)) {
-    const TcShape ts = tc_shape(c, m);
+    const TcShape ts = tc_shape(c, m, routed->gate.format);
     const TcLayout tl = tc_layout(c, m, base_layout_of(&c, m).total);
     const int sms = sm_count();
     if (sms <= 0) return MOE_ERR_UNSUPPORTED_DEVICE;
     tc::TcExtra tx;
     std::memset(&tx, 0, sizeof(tx));
-    tx.W = sms * tc::kWarps;
+    tx.W = sms * tc::kMaxWarps;
     const int split = g_forced_split.load(std::memory_order_relaxed);
     tx.gu_piece = ts.gu_slots && (split == 2 || (split == 0 && ts.j_gu_max < 4 * tx.W));
     // down jobs are split only when their rows come from HBM: when every active expert's down
@@ -741,6 +743,9 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
     pl.spin_limit = g_test_spin_limit.load() > 0 ? g_test_spin_limit.load() : kSpinLimit;
     pl.bar_extra = (unsigned)g_test_bar_extra.load();
     pl.l2_prefetch_cap = l2_cap;
+#ifdef MOE_NO_DOWN_PREFETCH
+    pl.l2_prefetch_cap = 0;  // measurement variant: no down-row prefetch into L2
+#endif
     const bool chain = forced_path() == 1;
     const int ntg = routed->gate.format == MOE_FMT_BF16 ? ts.ntg : (ts.ntg < 2 ? ts.ntg : 2);
     const cudaError_t e = tc_launch(routed->gate.format, ntg, chain, sms, st, p, tx, pl,

@@ -51,10 +51,13 @@
 namespace moe {
 namespace tc {
 
-constexpr int kChunk = 256;    // elements of K per canonical chunk
+// Elements of K per canonical chunk: about 16 KB of a 32-row job's weights in every format
+// (256 bf16, 512 FP8, 1024 4-bit elements). Fixed per format, whatever m.
+__host__ __device__ constexpr int chunk_elems(int fmt) {
+  return fmt == MOE_FMT_BF16 ? 256 : fmt == MOE_FMT_FP8_E4M3 ? 512 : 1024;
+}
 constexpr int kJobRows = 32;   // weight rows per job (two m16 tiles)
-constexpr int kThreads = 256;  // threads per CTA of every tensor-core kernel
-constexpr int kWarps = kThreads / 32;
+constexpr int kMaxWarps = 16;   // warps per CTA of a tensor-core kernel: 16 or 8 (below)
 constexpr int kMaxPairs = MOE_MAX_ROWS * MOE_MAX_TOP_K;  // 512
 constexpr unsigned kOnes = 0x3C003C00u;  // fp16 pair (1, 1)
 
@@ -101,7 +104,7 @@ constexpr bool tc_format() {
 }
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
-__host__ __device__ constexpr int n_chunks(int K) { return ceil_div(K, kChunk); }
+__host__ __device__ constexpr int n_chunks(int K, int fmt) { return ceil_div(K, chunk_elems(fmt)); }
 
 // Position of element i of a row in this library's stored activation order (Q4: a 4x4 transpose
 // inside every 16 elements, so a lane's k-step reads 4 consecutive stored elements).
@@ -418,10 +421,7 @@ struct SlotMap {
 // the scale words [u][row][word][lane] (the 4-byte aligned word holding the lane's scale bytes),
 // and the activation pieces [u][k-step pair (HILO: k-step)][live column][t] (16 bytes each) of
 // the lane's live columns only. kStages stages are in flight.
-constexpr int kRingBytes = 24 * 1024;  // per warp
-constexpr int kStages = 4;
-constexpr int kStageBytes = kRingBytes / kStages;
-constexpr int kRingWarpsBytes = kRingBytes * kWarps;  // dynamic shared memory per CTA
+constexpr int kRingCtaBytes = 192 * 1024;  // dynamic shared memory per CTA: the warps' rings
 
 __device__ __forceinline__ void cp16_ef(uint32_t dst, const void* src, int n, uint64_t pol) {
   asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst),
@@ -458,6 +458,32 @@ constexpr int scale_words() {  // aligned scale words per (row, k-tile)
   return FMT == MOE_FMT_Q4_AFFINE_G64 ? 2 : (FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_MXFP4) ? 1 : 0;
 }
 
+// Ring bytes one k-tile takes with `cols` live activation columns.
+template <int FMT, bool HILO>
+__host__ __device__ constexpr int ring_per_kt(int cols) {
+  return 128 * Traits<FMT>::BPL + 128 * 4 * scale_words<FMT>() +
+         (HILO ? Traits<FMT>::KS : Traits<FMT>::KS / 2) * cols * 64;
+}
+
+// Warps per CTA: 16 when each warp's share of the ring still holds two stages of a k-tile with
+// every column live (and one column group is 8 wide), else 8. More warps hide more latency.
+template <int FMT, int NTG>
+__host__ __device__ constexpr int tc_warps() {
+  return NTG == 1 && 2 * ring_per_kt<FMT, true>(8) <= kRingCtaBytes / 16 ? 16 : 8;
+}
+template <int FMT, int NTG>
+__host__ __device__ constexpr int ring_bytes() {
+  return kRingCtaBytes / tc_warps<FMT, NTG>();
+}
+
+// Stages of the ring: as many (2 to 4) as hold a k-tile with every column of the group live.
+template <int FMT, int NTG, bool HILO>
+constexpr int ring_stages() {
+  constexpr int n = ring_bytes<FMT, NTG>() / ring_per_kt<FMT, HILO>(8 * NTG);
+  static_assert(n >= 2, "a ring stage must hold one k-tile of every live column");
+  return n > 4 ? 4 : n;
+}
+
 // Address of the scale bytes a lane needs for row r, k-tile kt (word w: Q4 0 = scale, 1 = bias).
 template <int FMT>
 __device__ __forceinline__ const uint8_t* scale_addr(const JobRows& R, int r, int kt, int t,
@@ -467,26 +493,30 @@ __device__ __forceinline__ const uint8_t* scale_addr(const JobRows& R, int r, in
   return (w == 0 ? R.sc[r] : R.bi[r]) + (size_t)kt * 2;
 }
 
-// Chunks [c0, c1) of a job (element range [c0 * 256, min(c1 * 256, K))). With sm.base null the
+// Chunks [c0, c1) of a job (elements [c0 * chunk, min(c1 * chunk, K))). With sm.base null the
 // chunk values are added to acc in order (the warp owns the whole job); otherwise each chunk's
-// values are stored where sm says. ring: this warp's kRingBytes of shared memory.
+// values are stored where sm says. ring: this warp's share of the CTA's ring memory.
 template <int FMT, int NTG, bool HILO>
 __device__ void run_chunks(const JobRows& R, const JobCols<NTG>& C, int ncols, int K, int c0,
                            int c1, float (&acc)[2][NTG][4], const SlotMap& sm, uint8_t* ring,
                            const void* dummy) {
   using Tr = Traits<FMT>;
   constexpr int KT = 4 * Tr::EPL;            // elements per k-tile
-  constexpr int TPC = kChunk / KT;           // k-tiles per chunk
+  constexpr int TPC = chunk_elems(FMT) / KT;  // k-tiles per chunk
   constexpr int SW = scale_words<FMT>();
   constexpr int KSB = HILO ? Tr::KS : Tr::KS / 2;  // 16-byte activation pieces per k-tile
+  constexpr int kStages = ring_stages<FMT, NTG, HILO>();
+  constexpr int kStageBytes = ring_bytes<FMT, NTG>() / kStages;
   const int lane = threadIdx.x & 31, t = lane & 3, g = lane >> 2;
   const int nkt = ceil_div(K, KT);
   const int kt_begin = c0 * TPC, kt_end = min(nkt, c1 * TPC);
-  // stage layout for this piece (ncols = live columns of this column group, <= 8 * NTG)
+  // stage layout for this piece (ncols = live columns of this column group, <= 8 * NTG): U
+  // k-tiles of ring_per_kt(ncols) <= kStageBytes bytes each (ring_stages guarantees U >= 1)
   const int a_bytes = 128 * Tr::BPL, s_bytes = 128 * 4 * SW, b_bytes = KSB * ncols * 64;
   const int per_kt = a_bytes + s_bytes + b_bytes;
+  if (ncols < 1 || ncols > 8 * NTG || per_kt > kStageBytes) return;  // unreachable by design
   int U = kStageBytes / per_kt;
-  U = U < 1 ? 1 : U > 8 ? 8 : U;
+  U = U > 8 ? 8 : U;
   const int s_off = U * a_bytes, b_off = U * (a_bytes + s_bytes);
   const int nb = ceil_div(kt_end - kt_begin, U);
   const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
@@ -858,30 +888,44 @@ __device__ void build_map(int nslots, bool piece, ItemsOf items_of, NchOf nch_of
   }
 }
 
-// f(slot, item, c0, c1, whole) for every unit range of this warp (one item at a time).
+// The units of CTA cta of G: the range [cta C / G, (cta+1) C / G) of the concatenated list, taken
+// by the CTA's warps `grab` units at a time from a shared-memory counter (zeroed before the
+// phase), so the warps of a CTA balance among themselves. f(slot, item, c0, c1, whole) runs one
+// piece (one item's chunks [c0, c1)).
 template <typename NchOf, typename PieceFn>
-__device__ __forceinline__ void for_units(const PhaseMap& pm, int nslots, int wid, int W,
-                                          bool piece, NchOf nch_of, PieceFn f) {
+__device__ __forceinline__ void for_units(const PhaseMap& pm, int nslots, int cta, int G,
+                                          bool piece, int warps, int* counter, NchOf nch_of,
+                                          PieceFn f) {
   const long long C = pm.unit_pre[nslots];
-  const int q0 = (int)((long long)wid * C / W), q1 = (int)((long long)(wid + 1) * C / W);
+  const int q0 = (int)((long long)cta * C / G), q1 = (int)((long long)(cta + 1) * C / G);
+  // about three grabs per warp: pieces stay long, the tail stays short
+  const int grab = piece ? max(1, (q1 - q0) / (3 * warps)) : 1;
   int a = 0;
-  int q = q0;
-  while (q < q1) {
-    while (pm.unit_pre[a + 1] <= q) ++a;
-    const int nch = nch_of(a);
-    const int per = piece ? nch : 1;
-    const int r = q - pm.unit_pre[a];
-    const int item = r / per;
-    if (!piece) {
-      f(a, item, 0, nch, true);
-      ++q;
-      continue;
+  for (;;) {
+    int u0 = 0;
+    if ((threadIdx.x & 31) == 0) u0 = atomicAdd(counter, grab);
+    u0 = q0 + __shfl_sync(0xffffffffu, u0, 0);
+    if (u0 >= q1) break;
+    const int u1 = min(u0 + grab, q1);
+    int q = u0;
+    while (pm.unit_pre[a] > q) --a;
+    while (q < u1) {
+      while (pm.unit_pre[a + 1] <= q) ++a;
+      const int nch = nch_of(a);
+      const int per = piece ? nch : 1;
+      const int r = q - pm.unit_pre[a];
+      const int item = r / per;
+      if (!piece) {
+        f(a, item, 0, nch, true);
+        ++q;
+        continue;
+      }
+      const int c = r - item * per;
+      const int item_end = pm.unit_pre[a] + (item + 1) * per;
+      const int c1 = c + ((u1 < item_end ? u1 : item_end) - q);
+      f(a, item, c, c1, c == 0 && c1 == nch);
+      q += c1 - c;
     }
-    const int c = r - item * per;
-    const int item_end = pm.unit_pre[a] + (item + 1) * per;
-    const int c1 = c + ((q1 < item_end ? q1 : item_end) - q);
-    f(a, item, c, c1, c == 0 && c1 == nch);
-    q += c1 - c;
   }
 }
 
@@ -924,11 +968,12 @@ __device__ void build_maps(const Params& p, const TcExtra& tx, const SlotView& s
 
 template <int FMT, int NTG>
 __device__ void gate_up_phase(const Params& p, const TcExtra& tx, const SlotView& sv,
-                              const PhaseMap& pm, int wid, uint8_t* ring) {
+                              const PhaseMap& pm, int* counter, uint8_t* ring) {
   constexpr bool F16 = Traits<FMT>::F16;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int U = sv.U, ns = U + p.has_shared;
-  for_units(pm, ns, wid, tx.W, tx.gu_piece != 0, [&](int) { return tx.nch_h; },
+  for_units(pm, ns, blockIdx.x, gridDim.x, tx.gu_piece != 0, tc_warps<FMT, NTG>(), counter,
+            [&](int) { return tx.nch_h; },
             [&](int a, int item, int c0, int c1, bool whole) {
     const bool sh = a == U;
     const int n = slot_cols(p, sv, a);
@@ -1006,7 +1051,7 @@ __device__ void gate_up_phase(const Params& p, const TcExtra& tx, const SlotView
 
 template <int FMT, int NTG>
 __device__ void down_phase(const Params& p, const TcExtra& tx, const SlotView& sv,
-                           const PhaseMap& pm, int wid, uint8_t* ring) {
+                           const PhaseMap& pm, int* counter, uint8_t* ring) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int U = sv.U, ns = U + p.has_shared;
   // (slot, column group) items per column tile: the blend waits for all of them
@@ -1014,7 +1059,8 @@ __device__ void down_phase(const Params& p, const TcExtra& tx, const SlotView& s
   for (int a = lane; a < ns; a += 32) col_target += (unsigned)ceil_div(slot_cols(p, sv, a), 8 * NTG);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) col_target += __shfl_xor_sync(0xffffffffu, col_target, o);
-  for_units(pm, ns, wid, tx.W, tx.dn_piece != 0, [&](int a) { return a == U ? tx.nch_s : tx.nch_i; },
+  for_units(pm, ns, blockIdx.x, gridDim.x, tx.dn_piece != 0, tc_warps<FMT, NTG>(), counter,
+            [&](int a) { return a == U ? tx.nch_s : tx.nch_i; },
             [&](int a, int item, int c0, int c1, bool whole) {
     const bool sh = a == U;
     const int n = slot_cols(p, sv, a);
@@ -1181,13 +1227,15 @@ struct TcPlan {
 //   D  gate/up jobs over all warps of the grid (tc::gate_up_phase); arrive and wait at barrier 2.
 //   E  down jobs over all warps; the warp completing a 32-column tile blends it (tc::down_phase).
 template <int FMT, int NTG>
-__global__ void __launch_bounds__(kThreads, 1) tc_fused_kernel(
+__global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_fused_kernel(
     const __grid_constant__ Params p, const __grid_constant__ TcExtra tx,
     const __grid_constant__ TcPlan pl) {
   extern __shared__ __align__(16) uint8_t tc_ring[];
+  constexpr int kWarps = tc_warps<FMT, NTG>(), kThreads = 32 * kWarps;
   __shared__ TcRoute R;
   __shared__ PhaseMap s_gu, s_dn;
   __shared__ unsigned long long s_base;
+  __shared__ int s_next[2];  // units taken so far by this CTA's warps in phases D and E
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const int m = p.m, k = p.k, te = m * k;
@@ -1206,7 +1254,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fused_kernel(
   pdl_wait();
   TC_STAMP(1);
   unsigned long long* bar_ctr = reinterpret_cast<unsigned long long*>(p.ctrl + kBarCounter);
-  if (tid == 0) s_base = ld_acquire_u64(bar_ctr) / (unsigned long long)G * (unsigned long long)G;
+  if (tid == 0) {
+    s_base = ld_acquire_u64(bar_ctr) / (unsigned long long)G * (unsigned long long)G;
+    s_next[0] = 0;
+    s_next[1] = 0;
+  }
   if (p.has_bias)
     for (int e = tid; e < p.E; e += kThreads) R.bias[e] = __ldg(p.expert_bias + e);
 
@@ -1292,7 +1344,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fused_kernel(
   __syncthreads();
 
   // ---- D: gate/up -------------------------------------------------------------------------------
-  gate_up_phase<FMT, NTG>(p, tx, sv, s_gu, wid, tc_ring + warp * kRingBytes);
+  gate_up_phase<FMT, NTG>(p, tx, sv, s_gu, &s_next[0], tc_ring + warp * ring_bytes<FMT, NTG>());
 #ifdef MOE_PHASE_TIMERS
   __syncthreads();
 #endif
@@ -1321,7 +1373,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_fused_kernel(
   pdl_launch_dependents();
 
   // ---- E: down + blend ------------------------------------------------------------------------
-  down_phase<FMT, NTG>(p, tx, sv, s_dn, wid, tc_ring + warp * kRingBytes);
+  down_phase<FMT, NTG>(p, tx, sv, s_dn, &s_next[1], tc_ring + warp * ring_bytes<FMT, NTG>());
 #ifdef MOE_PHASE_TIMERS
   __syncthreads();
 #endif
@@ -1408,33 +1460,37 @@ __device__ __forceinline__ SlotView global_slots(const Params& p, const int* slo
 }
 
 template <int FMT, int NTG>
-__global__ void __launch_bounds__(kThreads, 1) tc_gate_up_kernel(
+__global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_gate_up_kernel(
     const __grid_constant__ Params p, const __grid_constant__ TcExtra tx, const int* slot_beg,
     const int* slot_n) {
   extern __shared__ __align__(16) uint8_t tc_ring[];
   __shared__ PhaseMap s_gu, s_dn;
+  __shared__ int s_next;
   pdl_launch_dependents();
   pdl_wait();
   const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) s_next = 0;
   const SlotView sv = global_slots(p, slot_beg, slot_n);
   build_maps<NTG>(p, tx, sv, s_gu, s_dn, warp);
   __syncthreads();
-  gate_up_phase<FMT, NTG>(p, tx, sv, s_gu, blockIdx.x * kWarps + warp, tc_ring + warp * kRingBytes);
+  gate_up_phase<FMT, NTG>(p, tx, sv, s_gu, &s_next, tc_ring + warp * ring_bytes<FMT, NTG>());
 }
 
 template <int FMT, int NTG>
-__global__ void __launch_bounds__(kThreads, 1) tc_down_kernel(
+__global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_down_kernel(
     const __grid_constant__ Params p, const __grid_constant__ TcExtra tx, const int* slot_beg,
     const int* slot_n) {
   extern __shared__ __align__(16) uint8_t tc_ring[];
   __shared__ PhaseMap s_gu, s_dn;
+  __shared__ int s_next;
   pdl_launch_dependents();
   pdl_wait();
   const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) s_next = 0;
   const SlotView sv = global_slots(p, slot_beg, slot_n);
   build_maps<NTG>(p, tx, sv, s_gu, s_dn, warp);
   __syncthreads();
-  down_phase<FMT, NTG>(p, tx, sv, s_dn, blockIdx.x * kWarps + warp, tc_ring + warp * kRingBytes);
+  down_phase<FMT, NTG>(p, tx, sv, s_dn, &s_next, tc_ring + warp * ring_bytes<FMT, NTG>());
 }
 
 }  // namespace tc
