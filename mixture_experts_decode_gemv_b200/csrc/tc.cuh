@@ -51,10 +51,16 @@
 namespace moe {
 namespace tc {
 
-// Elements of K per canonical chunk: about 16 KB of a 32-row job's weights in every format
-// (256 bf16, 512 FP8, 1024 4-bit elements). Fixed per format, whatever m.
+// Elements of K per canonical chunk: eight k-tiles of the format (256 bf16, 512 FP8, 1024 NVFP4,
+// 256 MXFP4, 512 Q4 elements), so a chunk costs about the same instructions in every format and a
+// one-row call has as many chunk-sized pieces to spread over the warps as the shapes allow.
+// Fixed per format, whatever m.
 __host__ __device__ constexpr int chunk_elems(int fmt) {
-  return fmt == MOE_FMT_BF16 ? 256 : fmt == MOE_FMT_FP8_E4M3 ? 512 : 1024;
+  return fmt == MOE_FMT_BF16 ? 256
+         : fmt == MOE_FMT_FP8_E4M3 ? 512
+         : fmt == MOE_FMT_NVFP4 ? 1024
+         : fmt == MOE_FMT_MXFP4 ? 256
+                                : 512;
 }
 constexpr int kJobRows = 32;   // weight rows per job (two m16 tiles)
 constexpr int kMaxWarps = 16;   // warps per CTA of a tensor-core kernel: 16 or 8 (below)
@@ -770,24 +776,35 @@ struct TcExtra {
 };
 
 // Optional phase timestamps (library built with -DMOE_PHASE_TIMERS): thread 0 of every CTA
-// writes the SM cycle counter at phase boundaries (slot 15: %globaltimer at entry, to line the
-// CTAs up) into a region at the end of the workspace.
+// keeps %globaltimer (ns) at phase boundaries in shared memory and writes them at the end of the
+// kernel into a region at the end of the workspace (slot 15: the entry time).
 #ifdef MOE_PHASE_TIMERS
+// The timer read is predicated on the value a shared-memory atomic returns, so the assembler
+// cannot move it above the barrier or the work before it.
 #define TC_STAMP(slot)                                                                 \
   do {                                                                                 \
-    if (threadIdx.x == 0 && tx.stamps != nullptr) {                                    \
+    if (threadIdx.x == 0) {                                                            \
       unsigned long long t_;                                                           \
-      asm volatile("mov.u64 %0, %%clock64;" : "=l"(t_)::"memory");                     \
-      tx.stamps[blockIdx.x * 16 + (slot)] = t_;                                        \
+      const uint32_t a_ = (uint32_t)__cvta_generic_to_shared(&s_stamps[(slot)]);      \
+      asm volatile(                                                                    \
+          "{ .reg .pred p_; .reg .u32 v_; atom.shared.add.u32 v_, [%1], 0;"            \
+          " setp.ne.u32 p_, v_, 0xFFFFFFFF; mov.u64 %0, 0; @p_ mov.u64 %0, %%globaltimer; }" \
+          : "=l"(t_) : "r"(a_) : "memory");                                            \
+      s_stamps[(slot)] = t_;                                                           \
     }                                                                                  \
   } while (0)
 #define TC_STAMP_GLOBAL()                                                              \
   do {                                                                                 \
-    if (threadIdx.x == 0 && tx.stamps != nullptr) {                                    \
+    if (threadIdx.x == 0) {                                                            \
       unsigned long long t_;                                                           \
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_)::"memory");                 \
-      tx.stamps[blockIdx.x * 16 + 15] = t_;                                            \
+      s_stamps[15] = t_;                                                               \
     }                                                                                  \
+  } while (0)
+#define TC_STAMP_FLUSH()                                                               \
+  do {                                                                                 \
+    if (threadIdx.x < 16 && tx.stamps != nullptr)                                      \
+      tx.stamps[blockIdx.x * 16 + threadIdx.x] = s_stamps[threadIdx.x];                \
   } while (0)
 #else
 #define TC_STAMP(slot) \
@@ -795,6 +812,9 @@ struct TcExtra {
   } while (0)
 #define TC_STAMP_GLOBAL() \
   do {                    \
+  } while (0)
+#define TC_STAMP_FLUSH() \
+  do {                   \
   } while (0)
 #endif
 
@@ -1236,6 +1256,9 @@ __global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_fused_kernel(
   __shared__ PhaseMap s_gu, s_dn;
   __shared__ unsigned long long s_base;
   __shared__ int s_next[2];  // units taken so far by this CTA's warps in phases D and E
+#ifdef MOE_PHASE_TIMERS
+  __shared__ unsigned long long s_stamps[16];
+#endif
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const int m = p.m, k = p.k, te = m * k;
@@ -1342,9 +1365,11 @@ __global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_fused_kernel(
   sv.U = U;
   build_maps<NTG>(p, tx, sv, s_gu, s_dn, warp);
   __syncthreads();
+  TC_STAMP(12);
 
   // ---- D: gate/up -------------------------------------------------------------------------------
   gate_up_phase<FMT, NTG>(p, tx, sv, s_gu, &s_next[0], tc_ring + warp * ring_bytes<FMT, NTG>());
+  TC_STAMP(10);  // warp 0's own share done
 #ifdef MOE_PHASE_TIMERS
   __syncthreads();
 #endif
@@ -1374,10 +1399,15 @@ __global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_fused_kernel(
 
   // ---- E: down + blend ------------------------------------------------------------------------
   down_phase<FMT, NTG>(p, tx, sv, s_dn, &s_next[1], tc_ring + warp * ring_bytes<FMT, NTG>());
+  TC_STAMP(11);  // warp 0's own share done
 #ifdef MOE_PHASE_TIMERS
   __syncthreads();
 #endif
   TC_STAMP(8);
+#ifdef MOE_PHASE_TIMERS
+  __syncthreads();
+#endif
+  TC_STAMP_FLUSH();
 }
 
 // ---- the multi-kernel path: router, gate/up, down -------------------------------------------------
