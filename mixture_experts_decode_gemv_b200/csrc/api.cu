@@ -129,6 +129,9 @@ int n_tiles_c_of(int h) { return (h + kColsPerCta - 1) / kColsPerCta; }
 // Split jobs keep their chunk values in the workspace: 32 floats per (activation column, job
 // tile, chunk). A phase may split its jobs when that storage stays within this size.
 constexpr size_t kSlotCapBytes = 24u << 20;
+// Down rows of a call are asked into L2 during gate/up when they total at most this many bytes
+// (well inside the 126 MB L2, next to the gate/up stream passing through it).
+constexpr long long kDownPrefetchCap = 48LL << 20;
 
 // Everything the tensor-core regions and work split depend on, from (cfg, m) alone.
 struct TcShape {
@@ -713,16 +716,12 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
     std::memset(&tx, 0, sizeof(tx));
     tx.W = sms * tc::kMaxWarps;
     const int split = g_forced_split.load(std::memory_order_relaxed);
-    tx.gu_piece = ts.gu_slots && (split == 2 || (split == 0 && ts.j_gu_max < 4 * tx.W));
-    // down jobs are split only when their rows come from HBM: when every active expert's down
-    // rows fit the L2 prefetch (asked for during gate/up), whole jobs read them from L2 with
-    // fewer serial round trips
-    const size_t down_max = ((size_t)p.cap * packed_row_bytes(routed->down.format, c.moe_inter) +
-                             (has_shared ? packed_row_bytes(routed->down.format, p.S) : 0)) *
-                            (size_t)c.hidden;
-    const long long l2_cap = 48LL << 20;
-    tx.dn_piece = ts.dn_slots && (split == 2 || (split == 0 && ts.j_dn_max < 4 * tx.W &&
-                                                 down_max > (size_t)l2_cap));
+    // whether a phase splits its jobs by chunk is decided in the kernel from the call's routing
+    // (tc::split_jobs); here: whether it may (its chunk values fit the workspace and no test
+    // forces whole jobs), and whether a test forces the split
+    tx.gu_piece = ts.gu_slots && split != 1;
+    tx.dn_piece = ts.dn_slots && split != 1;
+    tx.force_split = split == 2;
     tx.tiles_i = ts.tiles_i;
     tx.tiles_s = ts.tiles_s;
     tx.tiles_h = ts.tiles_h;
@@ -742,10 +741,7 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
     tc::TcPlan pl;
     pl.spin_limit = g_test_spin_limit.load() > 0 ? g_test_spin_limit.load() : kSpinLimit;
     pl.bar_extra = (unsigned)g_test_bar_extra.load();
-    pl.l2_prefetch_cap = l2_cap;
-#ifdef MOE_NO_DOWN_PREFETCH
-    pl.l2_prefetch_cap = 0;  // measurement variant: no down-row prefetch into L2
-#endif
+    pl.l2_prefetch_cap = kDownPrefetchCap;
     const bool chain = forced_path() == 1;
     const int ntg = routed->gate.format == MOE_FMT_BF16 ? ts.ntg : (ts.ntg < 2 ? ts.ntg : 2);
     const cudaError_t e = tc_launch(routed->gate.format, ntg, chain, sms, st, p, tx, pl,

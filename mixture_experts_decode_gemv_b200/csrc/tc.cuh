@@ -757,8 +757,9 @@ struct SlotView {
 
 struct TcExtra {
   int W;               // warps taking part in a phase (all of the grid)
-  int gu_piece;        // 1: gate/up jobs are split by chunk; 0: whole jobs per warp
+  int gu_piece;        // 1: gate/up jobs may be split by chunk (their chunk values fit); 0: not
   int dn_piece;        // the same for down
+  int force_split;     // 1: split every phase that may split (tests); 0: the rule of split_jobs
   int tiles_i, tiles_s;  // gate/up jobs per routed / shared expert (16 row pairs each)
   int tiles_h;         // down jobs per expert (32 output columns each)
   int nch_h, nch_i, nch_s;  // chunks of h, I, S
@@ -875,7 +876,23 @@ __device__ void convert_x(const Params& p, const TcExtra& tx, int gtid, int nthr
 struct PhaseMap {
   int item_pre[kMaxPairs + 2];  // first item of each slot
   int unit_pre[kMaxPairs + 2];  // first unit of each slot
+  int piece;                    // 1: the phase's jobs are split by chunk
 };
+
+// Whether a phase of J jobs (items) runs split by chunk on a grid of W warps. Below a threshold
+// there are too few whole jobs to keep enough warps streaming: fewer than W for the 4-bit
+// formats (a k-tile costs many decode and scale instructions, so a warp's serial chain sets the
+// time), fewer than W / 2 for bf16 and FP8 (a k-tile is mostly its memory round trip, and every
+// piece restarts the warp's copy pipeline and adds a ticket). From there to W whole jobs keep
+// the grid busy. Above W, whole jobs are kept unless they leave the busiest warp more than 10%
+// above the average. Measured on the B200 with cold calls at m = 1..64 over the published shapes.
+__device__ __forceinline__ bool split_jobs(int J, int W, bool four_bit) {
+  if (J <= 0) return false;
+  if (J < (four_bit ? W : W / 2)) return true;
+  if (J < W) return false;
+  const long long per = (J + W - 1) / W;
+  return per * W * 10 > (long long)J * 11;
+}
 
 // By one warp: the prefix sums of a phase over nslots slots.
 template <typename ItemsOf, typename NchOf>
@@ -918,8 +935,9 @@ __device__ __forceinline__ void for_units(const PhaseMap& pm, int nslots, int ct
                                           PieceFn f) {
   const long long C = pm.unit_pre[nslots];
   const int q0 = (int)((long long)cta * C / G), q1 = (int)((long long)(cta + 1) * C / G);
-  // about three grabs per warp: pieces stay long, the tail stays short
-  const int grab = piece ? max(1, (q1 - q0) / (3 * warps)) : 1;
+  // split jobs: about one grab per warp, so pieces stay long (fewer pipeline restarts and
+  // tickets); a warp that finishes early takes what a late one has not
+  const int grab = piece ? max(1, (q1 - q0 + warps - 1) / warps) : 1;
   int a = 0;
   for (;;) {
     int u0 = 0;
@@ -967,20 +985,34 @@ __device__ __forceinline__ int slot_cols(const Params& p, const SlotView& sv, in
   return a == sv.U ? p.m : sv.slot_n[a];
 }
 
-// The prefix maps of both phases (one warp builds each).
-template <int NTG>
+// The prefix maps of both phases (one warp builds each), with each phase's split decision taken
+// from its job count (split_jobs) on this call's routing.
+template <int FMT, int NTG>
 __device__ void build_maps(const Params& p, const TcExtra& tx, const SlotView& sv, PhaseMap& gu,
                            PhaseMap& dn, int warp) {
+  constexpr bool kFourBit =
+      FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_MXFP4 || FMT == MOE_FMT_Q4_AFFINE_G64;
   const int ns = sv.U + p.has_shared;
+  const int W = gridDim.x * tc_warps<FMT, NTG>();
+  auto jobs = [&](auto items_of) {  // items of the phase, by one warp
+    int J = 0;
+    for (int a = threadIdx.x & 31; a < ns; a += 32) J += items_of(a);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) J += __shfl_xor_sync(0xffffffffu, J, o);
+    return J;
+  };
   if (warp == 0) {
-    build_map(ns, tx.gu_piece != 0,
-              [&](int a) { return (a == sv.U ? tx.tiles_s : tx.tiles_i) *
-                                  ceil_div(slot_cols(p, sv, a), 8 * NTG); },
-              [&](int) { return tx.nch_h; }, gu);
+    auto items = [&](int a) {
+      return (a == sv.U ? tx.tiles_s : tx.tiles_i) * ceil_div(slot_cols(p, sv, a), 8 * NTG);
+    };
+    const bool piece = tx.gu_piece != 0 && (tx.force_split != 0 || split_jobs(jobs(items), W, kFourBit));
+    build_map(ns, piece, items, [&](int) { return tx.nch_h; }, gu);
+    if ((threadIdx.x & 31) == 0) gu.piece = piece;
   } else if (warp == 1) {
-    build_map(ns, tx.dn_piece != 0,
-              [&](int a) { return tx.tiles_h * ceil_div(slot_cols(p, sv, a), 8 * NTG); },
-              [&](int a) { return a == sv.U ? tx.nch_s : tx.nch_i; }, dn);
+    auto items = [&](int a) { return tx.tiles_h * ceil_div(slot_cols(p, sv, a), 8 * NTG); };
+    const bool piece = tx.dn_piece != 0 && (tx.force_split != 0 || split_jobs(jobs(items), W, kFourBit));
+    build_map(ns, piece, items, [&](int a) { return a == sv.U ? tx.nch_s : tx.nch_i; }, dn);
+    if ((threadIdx.x & 31) == 0) dn.piece = piece;
   }
 }
 
@@ -992,7 +1024,7 @@ __device__ void gate_up_phase(const Params& p, const TcExtra& tx, const SlotView
   constexpr bool F16 = Traits<FMT>::F16;
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int U = sv.U, ns = U + p.has_shared;
-  for_units(pm, ns, blockIdx.x, gridDim.x, tx.gu_piece != 0, tc_warps<FMT, NTG>(), counter,
+  for_units(pm, ns, blockIdx.x, gridDim.x, pm.piece != 0, tc_warps<FMT, NTG>(), counter,
             [&](int) { return tx.nch_h; },
             [&](int a, int item, int c0, int c1, bool whole) {
     const bool sh = a == U;
@@ -1079,7 +1111,7 @@ __device__ void down_phase(const Params& p, const TcExtra& tx, const SlotView& s
   for (int a = lane; a < ns; a += 32) col_target += (unsigned)ceil_div(slot_cols(p, sv, a), 8 * NTG);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) col_target += __shfl_xor_sync(0xffffffffu, col_target, o);
-  for_units(pm, ns, blockIdx.x, gridDim.x, tx.dn_piece != 0, tc_warps<FMT, NTG>(), counter,
+  for_units(pm, ns, blockIdx.x, gridDim.x, pm.piece != 0, tc_warps<FMT, NTG>(), counter,
             [&](int a) { return a == U ? tx.nch_s : tx.nch_i; },
             [&](int a, int item, int c0, int c1, bool whole) {
     const bool sh = a == U;
@@ -1363,7 +1395,7 @@ __global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_fused_kernel(
   sv.tp = R.tp;
   sv.gamma = R.gamma;
   sv.U = U;
-  build_maps<NTG>(p, tx, sv, s_gu, s_dn, warp);
+  build_maps<FMT, NTG>(p, tx, sv, s_gu, s_dn, warp);
   __syncthreads();
   TC_STAMP(12);
 
@@ -1501,7 +1533,7 @@ __global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_gate_up_kerne
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) s_next = 0;
   const SlotView sv = global_slots(p, slot_beg, slot_n);
-  build_maps<NTG>(p, tx, sv, s_gu, s_dn, warp);
+  build_maps<FMT, NTG>(p, tx, sv, s_gu, s_dn, warp);
   __syncthreads();
   gate_up_phase<FMT, NTG>(p, tx, sv, s_gu, &s_next, tc_ring + warp * ring_bytes<FMT, NTG>());
 }
@@ -1518,7 +1550,7 @@ __global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_down_kernel(
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) s_next = 0;
   const SlotView sv = global_slots(p, slot_beg, slot_n);
-  build_maps<NTG>(p, tx, sv, s_gu, s_dn, warp);
+  build_maps<FMT, NTG>(p, tx, sv, s_gu, s_dn, warp);
   __syncthreads();
   down_phase<FMT, NTG>(p, tx, sv, s_dn, &s_next, tc_ring + warp * ring_bytes<FMT, NTG>());
 }
