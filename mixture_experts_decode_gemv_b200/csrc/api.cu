@@ -147,9 +147,15 @@ TcShape tc_shape(const moe_cfg& c, int m, int fmt = MOE_FMT_BF16) {
   TcShape t;
   const bool has_shared = c.shared_kind != MOE_SHARED_NONE;
   const int S = has_shared ? c.shared_inter : 0;
-  t.ntg = m <= 8 ? 1 : m <= 16 ? 2 : 4;   // n-tiles of 8 activation columns per pass (bf16;
-                                          // the other formats take at most 2)
-  t.ncg_max = tc::ceil_div(m, 8 * (t.ntg < 2 ? t.ntg : 2));  // column groups at the smallest width
+  // n-tiles of 8 activation columns per pass. One, so that a CTA runs as many warps as its
+  // format allows (16; 8 for NVFP4: more latency hidden, no MMAs on absent columns) even though a slot with many columns (the shared expert)
+  // then streams its weight tiles once per 8 columns, mostly from L2. Two for Q4 above 8 rows
+  // (its decode and post-scale work per weight byte is the largest) and for bf16 layers with a
+  // shared expert above 32 rows (a shared expert as large as Llama-4-Scout's, read 8 times
+  // from L2 per call, costs more than the smaller CTA). Measured on the B200 at m = 16..64.
+  const bool q4 = fmt == MOE_FMT_Q4_AFFINE_G64;
+  t.ntg = q4 ? (m <= 8 ? 1 : 2) : (fmt == MOE_FMT_BF16 && has_shared && m > 32) ? 2 : 1;
+  t.ncg_max = tc::ceil_div(m, 8);  // column groups at the smallest width (any format)
   t.tiles_i = tc::ceil_div(c.moe_inter, 16);
   t.tiles_s = S ? tc::ceil_div(S, 16) : 0;
   t.tiles_h = tc::ceil_div(c.hidden, 32);
@@ -572,9 +578,6 @@ cudaError_t tc_run(bool chain, int sms, cudaStream_t st, const Params& p, const 
 template <int FMT>
 cudaError_t tc_run_ntg(int ntg, bool chain, int sms, cudaStream_t st, const Params& p,
                        const tc::TcExtra& tx, const tc::TcPlan& pl, int* sb, int* sn) {
-  if constexpr (FMT == MOE_FMT_BF16) {
-    if (ntg == 4) return tc_run<FMT, 4>(chain, sms, st, p, tx, pl, sb, sn);
-  }
   return ntg == 1 ? tc_run<FMT, 1>(chain, sms, st, p, tx, pl, sb, sn)
                   : tc_run<FMT, 2>(chain, sms, st, p, tx, pl, sb, sn);
 }
@@ -743,7 +746,7 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
     pl.bar_extra = (unsigned)g_test_bar_extra.load();
     pl.l2_prefetch_cap = kDownPrefetchCap;
     const bool chain = forced_path() == 1;
-    const int ntg = routed->gate.format == MOE_FMT_BF16 ? ts.ntg : (ts.ntg < 2 ? ts.ntg : 2);
+    const int ntg = ts.ntg;
     const cudaError_t e = tc_launch(routed->gate.format, ntg, chain, sms, st, p, tx, pl,
                                     (int*)(ws + tl.slot_beg), (int*)(ws + tl.slot_n));
     if (e != cudaSuccess) return cuda_fail(e);

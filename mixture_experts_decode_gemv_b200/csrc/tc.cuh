@@ -426,7 +426,7 @@ struct SlotMap {
 // synchronisation. A stage holds U k-tiles: the weight pieces [u][row][lane] (BPL bytes each),
 // the scale words [u][row][word][lane] (the 4-byte aligned word holding the lane's scale bytes),
 // and the activation pieces [u][k-step pair (HILO: k-step)][live column][t] (16 bytes each) of
-// the lane's live columns only. kStages stages are in flight.
+// the lane's live columns only. 2 to 8 stages, as many as the job's live columns leave room for.
 constexpr int kRingCtaBytes = 192 * 1024;  // dynamic shared memory per CTA: the warps' rings
 
 __device__ __forceinline__ void cp16_ef(uint32_t dst, const void* src, int n, uint64_t pol) {
@@ -458,6 +458,18 @@ template <int N>
 __device__ __forceinline__ void cp_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// cp_wait with a count known only at run time (1..7; warp-uniform)
+__device__ __forceinline__ void cp_wait_n(int n) {
+  switch (n) {
+    case 1: cp_wait<1>(); break;
+    case 2: cp_wait<2>(); break;
+    case 3: cp_wait<3>(); break;
+    case 4: cp_wait<4>(); break;
+    case 5: cp_wait<5>(); break;
+    case 6: cp_wait<6>(); break;
+    default: cp_wait<7>(); break;
+  }
+}
 
 template <int FMT>
 constexpr int scale_words() {  // aligned scale words per (row, k-tile)
@@ -482,12 +494,10 @@ __host__ __device__ constexpr int ring_bytes() {
   return kRingCtaBytes / tc_warps<FMT, NTG>();
 }
 
-// Stages of the ring: as many (2 to 4) as hold a k-tile with every column of the group live.
+// k-tiles with every column of the group live that a warp's ring holds (at least 2 are needed).
 template <int FMT, int NTG, bool HILO>
 constexpr int ring_stages() {
-  constexpr int n = ring_bytes<FMT, NTG>() / ring_per_kt<FMT, HILO>(8 * NTG);
-  static_assert(n >= 2, "a ring stage must hold one k-tile of every live column");
-  return n > 4 ? 4 : n;
+  return ring_bytes<FMT, NTG>() / ring_per_kt<FMT, HILO>(8 * NTG);
 }
 
 // Address of the scale bytes a lane needs for row r, k-tile kt (word w: Q4 0 = scale, 1 = bias).
@@ -511,18 +521,23 @@ __device__ void run_chunks(const JobRows& R, const JobCols<NTG>& C, int ncols, i
   constexpr int TPC = chunk_elems(FMT) / KT;  // k-tiles per chunk
   constexpr int SW = scale_words<FMT>();
   constexpr int KSB = HILO ? Tr::KS : Tr::KS / 2;  // 16-byte activation pieces per k-tile
-  constexpr int kStages = ring_stages<FMT, NTG, HILO>();
-  constexpr int kStageBytes = ring_bytes<FMT, NTG>() / kStages;
+  constexpr int kRing = ring_bytes<FMT, NTG>();
+  static_assert(ring_stages<FMT, NTG, HILO>() >= 2, "the ring must hold two widest k-tiles");
   const int lane = threadIdx.x & 31, t = lane & 3, g = lane >> 2;
   const int nkt = ceil_div(K, KT);
   const int kt_begin = c0 * TPC, kt_end = min(nkt, c1 * TPC);
   // stage layout for this piece (ncols = live columns of this column group, <= 8 * NTG): U
-  // k-tiles of ring_per_kt(ncols) <= kStageBytes bytes each (ring_stages guarantees U >= 1)
+  // k-tiles of per_kt bytes per stage, U as large as keeps at least four stages (at most 8
+  // k-tiles), then as many stages as the ring holds (2 to 8): the fewer live columns, the more
+  // weight bytes in flight
   const int a_bytes = 128 * Tr::BPL, s_bytes = 128 * 4 * SW, b_bytes = KSB * ncols * 64;
   const int per_kt = a_bytes + s_bytes + b_bytes;
-  if (ncols < 1 || ncols > 8 * NTG || per_kt > kStageBytes) return;  // unreachable by design
-  int U = kStageBytes / per_kt;
-  U = U > 8 ? 8 : U;
+  if (ncols < 1 || ncols > 8 * NTG || 2 * per_kt > kRing) return;  // unreachable by design
+  int U = kRing / (4 * per_kt);
+  U = U < 1 ? 1 : U > 8 ? 8 : U;
+  int S = kRing / (U * per_kt);
+  S = S > 8 ? 8 : S;
+  const int SB = U * per_kt;  // a multiple of 16 bytes
   const int s_off = U * a_bytes, b_off = U * (a_bytes + s_bytes);
   const int nb = ceil_div(kt_end - kt_begin, U);
   const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
@@ -532,7 +547,7 @@ __device__ void run_chunks(const JobRows& R, const JobCols<NTG>& C, int ncols, i
   for (int q = 0; q < NTG; ++q) cidx[q] = (C.row[q] != nullptr) ? 8 * q + g : -1;
 
   auto issue = [&](int b) {
-    const uint32_t st = ring_s + (uint32_t)((b % kStages) * kStageBytes);
+    const uint32_t st = ring_s + (uint32_t)((b % S) * SB);
     for (int u = 0; u < U; ++u) {
       const int kt = kt_begin + b * U + u;
       if (kt >= kt_end) break;
@@ -588,16 +603,17 @@ __device__ void run_chunks(const JobRows& R, const JobCols<NTG>& C, int ncols, i
   float d1[NTG][4];     // Q4: the all-ones chain
   zero<NTG>(p);
   zero<NTG>(d);
-#pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
+  for (int s = 0; s < S - 1; ++s) {
     if (s < nb) issue(s);
     cp_commit();
   }
+  int rd = 0;  // stage of batch b
   for (int b = 0; b < nb; ++b) {
-    if (b + kStages - 1 < nb) issue(b + kStages - 1);
+    if (b + S - 1 < nb) issue(b + S - 1);
     cp_commit();
-    cp_wait<kStages - 1>();  // this lane's copies of batch b have landed
-    const uint8_t* st = ring + (b % kStages) * kStageBytes;
+    cp_wait_n(S - 1);  // this lane's copies of batch b have landed
+    const uint8_t* st = ring + rd * SB;
+    rd = rd + 1 == S ? 0 : rd + 1;
     for (int u = 0; u < U; ++u) {
       const int kt = kt_begin + b * U + u;
       if (kt >= kt_end) break;  // warp-uniform
@@ -925,20 +941,35 @@ __device__ void build_map(int nslots, bool piece, ItemsOf items_of, NchOf nch_of
   }
 }
 
-// The units of CTA cta of G: the range [cta C / G, (cta+1) C / G) of the concatenated list, taken
-// by the CTA's warps `grab` units at a time from a shared-memory counter (zeroed before the
-// phase), so the warps of a CTA balance among themselves. f(slot, item, c0, c1, whole) runs one
-// piece (one item's chunks [c0, c1)).
+// The units of CTA cta of G, taken by the CTA's warps from a shared-memory counter (zeroed before
+// the phase), so the warps of a CTA balance among themselves. Split jobs: the range
+// [cta C / G, (cta+1) C / G) of the concatenated list, `grab` units at a time, so that a piece
+// covers consecutive chunks. Whole jobs: every G-th job from cta on, so that every CTA gets its
+// share of each slot's jobs (jobs of a slot with many live columns stream fewer weight bytes per
+// ring stage, and a contiguous range would give them all to the last CTAs).
+// f(slot, item, c0, c1, whole) runs one piece (one item's chunks [c0, c1)).
 template <typename NchOf, typename PieceFn>
 __device__ __forceinline__ void for_units(const PhaseMap& pm, int nslots, int cta, int G,
                                           bool piece, int warps, int* counter, NchOf nch_of,
                                           PieceFn f) {
   const long long C = pm.unit_pre[nslots];
+  int a = 0;
+  if (!piece) {
+    for (;;) {
+      int k = 0;
+      if ((threadIdx.x & 31) == 0) k = atomicAdd(counter, 1);
+      k = __shfl_sync(0xffffffffu, k, 0);
+      const long long q = cta + (long long)k * G;
+      if (q >= C) break;
+      while (pm.unit_pre[a + 1] <= q) ++a;
+      f(a, (int)(q - pm.unit_pre[a]), 0, nch_of(a), true);
+    }
+    return;
+  }
   const int q0 = (int)((long long)cta * C / G), q1 = (int)((long long)(cta + 1) * C / G);
   // split jobs: about one grab per warp, so pieces stay long (fewer pipeline restarts and
   // tickets); a warp that finishes early takes what a late one has not
-  const int grab = piece ? max(1, (q1 - q0 + warps - 1) / warps) : 1;
-  int a = 0;
+  const int grab = max(1, (q1 - q0 + warps - 1) / warps);
   for (;;) {
     int u0 = 0;
     if ((threadIdx.x & 31) == 0) u0 = atomicAdd(counter, grab);
@@ -950,14 +981,9 @@ __device__ __forceinline__ void for_units(const PhaseMap& pm, int nslots, int ct
     while (q < u1) {
       while (pm.unit_pre[a + 1] <= q) ++a;
       const int nch = nch_of(a);
-      const int per = piece ? nch : 1;
+      const int per = nch;
       const int r = q - pm.unit_pre[a];
       const int item = r / per;
-      if (!piece) {
-        f(a, item, 0, nch, true);
-        ++q;
-        continue;
-      }
       const int c = r - item * per;
       const int item_end = pm.unit_pre[a] + (item + 1) * per;
       const int c1 = c + ((u1 < item_end ? u1 : item_end) - q);
