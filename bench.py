@@ -44,7 +44,10 @@ SWEEP_CONFIGS = ("qwen3_30b_a3b", "lfm2_8b_a1b", "qwen3_6_35b_a3b", "llama4_scou
 # DRAM bytes per call (dram__bytes_read.sum + dram__bytes_write.sum summed over the call's
 # launches, one ncu capture of the current kernels; the summaries are in profiles/). Keyed by
 # (workload config name, m); entries are removed whenever the kernels they measured change.
-PROFILED_TRAFFIC: dict = {}
+# DRAM bytes (read + write) per launch of the layer's kernel, from a single-pass ncu capture of
+# the same workload (profiles/tc_fused_kernel_traffic_llama4_scout_m64.md); retaken whenever the
+# kernel changes.
+PROFILED_TRAFFIC: dict = {("llama4_scout", 64): 4.03e9 + 5.9e6}
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 WINDOWS = 5

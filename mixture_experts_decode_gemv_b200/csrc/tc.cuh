@@ -546,8 +546,8 @@ __device__ void run_chunks(const JobRows& R, const JobCols<NTG>& C, int ncols, i
 #pragma unroll
   for (int q = 0; q < NTG; ++q) cidx[q] = (C.row[q] != nullptr) ? 8 * q + g : -1;
 
-  auto issue = [&](int b) {
-    const uint32_t st = ring_s + (uint32_t)((b % S) * SB);
+  auto issue = [&](int b, int stage) {
+    const uint32_t st = ring_s + (uint32_t)(stage * SB);
     for (int u = 0; u < U; ++u) {
       const int kt = kt_begin + b * U + u;
       if (kt >= kt_end) break;
@@ -604,12 +604,13 @@ __device__ void run_chunks(const JobRows& R, const JobCols<NTG>& C, int ncols, i
   zero<NTG>(p);
   zero<NTG>(d);
   for (int s = 0; s < S - 1; ++s) {
-    if (s < nb) issue(s);
+    if (s < nb) issue(s, s);
     cp_commit();
   }
-  int rd = 0;  // stage of batch b
+  int rd = 0, wr = S - 1;  // stages of batch b and of batch b + S - 1
   for (int b = 0; b < nb; ++b) {
-    if (b + S - 1 < nb) issue(b + S - 1);
+    if (b + S - 1 < nb) issue(b + S - 1, wr);
+    wr = wr + 1 == S ? 0 : wr + 1;
     cp_commit();
     cp_wait_n(S - 1);  // this lane's copies of batch b have landed
     const uint8_t* st = ring + rd * SB;
@@ -906,8 +907,8 @@ __device__ __forceinline__ bool split_jobs(int J, int W, bool four_bit) {
   if (J <= 0) return false;
   if (J < (four_bit ? W : W / 2)) return true;
   if (J < W) return false;
-  const long long per = (J + W - 1) / W;
-  return per * W * 10 > (long long)J * 11;
+  const int per = (J + W - 1) / W;  // whole jobs of the busiest warp
+  return (long long)per * W * 10 > (long long)J * 11;
 }
 
 // By one warp: the prefix sums of a phase over nslots slots.
@@ -1421,7 +1422,9 @@ __global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_fused_kernel(
   sv.tp = R.tp;
   sv.gamma = R.gamma;
   sv.U = U;
+  TC_STAMP(13);
   build_maps<FMT, NTG>(p, tx, sv, s_gu, s_dn, warp);
+  TC_STAMP(14);
   __syncthreads();
   TC_STAMP(12);
 
