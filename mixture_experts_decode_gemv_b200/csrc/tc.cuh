@@ -741,19 +741,36 @@ __device__ void run_chunks(const JobRows& R, const JobCols<NTG>& C, int ncols, i
 template <int NTG>
 __device__ __forceinline__ void sum_slots(const SlotMap& sm, int nch, float (&acc)[2][NTG][4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  constexpr int kB = NTG == 1 ? 4 : 2;  // chunks whose values are loaded together
   zero<NTG>(acc);
-  for (int c = 0; c < nch; ++c) {
+  for (int c0 = 0; c0 < nch; c0 += kB) {
+    // every load of the batch first (one round trip to L2), then the adds in chunk order
+    float v[kB][2][NTG][4];
 #pragma unroll
-    for (int m = 0; m < 2; ++m)
+    for (int b = 0; b < kB; ++b)
 #pragma unroll
-      for (int n = 0; n < NTG; ++n)
+      for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int col = sm.col0 + 8 * n + 2 * t + (q & 1);
-          const int r = 16 * m + g + (q >= 2 ? 8 : 0);
-          if (col < sm.n)
-            acc[m][n][q] += __ldcg(sm.base + (size_t)col * sm.col_stride + (size_t)c * 32 + r);
-        }
+        for (int n = 0; n < NTG; ++n)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int col = sm.col0 + 8 * n + 2 * t + (q & 1);
+            const int r = 16 * m + g + (q >= 2 ? 8 : 0);
+            v[b][m][n][q] = (col < sm.n && c0 + b < nch)
+                                ? __ldcg(sm.base + (size_t)col * sm.col_stride +
+                                         (size_t)(c0 + b) * 32 + r)
+                                : 0.f;
+          }
+#pragma unroll
+    for (int b = 0; b < kB; ++b) {
+      if (c0 + b >= nch) break;
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int n = 0; n < NTG; ++n)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[m][n][q] += v[b][m][n][q];
+    }
   }
 }
 
@@ -911,34 +928,45 @@ __device__ __forceinline__ bool split_jobs(int J, int W, bool four_bit) {
   return (long long)per * W * 10 > (long long)J * 11;
 }
 
-// By one warp: the prefix sums of a phase over nslots slots.
-template <typename ItemsOf, typename NchOf>
-__device__ void build_map(int nslots, bool piece, ItemsOf items_of, NchOf nch_of, PhaseMap& pm) {
+// By one warp: the prefix map of a phase over nslots slots. One scan gives the items (jobs)
+// before each slot and their total J, from which decide(J) says whether the phase splits its jobs
+// by chunk; the units before slot a are then its items times the chunks per job (nch_a for every
+// slot but the last, which has nch_last: the shared expert's down jobs may differ).
+template <typename ItemsOf, typename Decide>
+__device__ void build_map(int nslots, int nch_a, int nch_last, ItemsOf items_of, Decide decide,
+                          PhaseMap& pm) {
   const int lane = threadIdx.x & 31;
-  int ib = 0, ub = 0;
+  int ib = 0, last_items = 0;
   for (int a0 = 0; a0 < nslots; a0 += 32) {
     const int a = a0 + lane;
     const int it = a < nslots ? items_of(a) : 0;
-    const int un = it * (piece && a < nslots ? nch_of(a) : 1);
-    int iti = it, uni = un;
+    int iti = it;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int x = __shfl_up_sync(0xffffffffu, iti, o), y = __shfl_up_sync(0xffffffffu, uni, o);
-      if (lane >= o) {
-        iti += x;
-        uni += y;
-      }
+      const int x = __shfl_up_sync(0xffffffffu, iti, o);
+      if (lane >= o) iti += x;
     }
-    if (a < nslots) {
-      pm.item_pre[a] = ib + iti - it;
-      pm.unit_pre[a] = ub + uni - un;
-    }
+    if (a < nslots) pm.item_pre[a] = ib + iti - it;
+    if (a == nslots - 1) last_items = it;
     ib += __shfl_sync(0xffffffffu, iti, 31);
-    ub += __shfl_sync(0xffffffffu, uni, 31);
+  }
+  last_items = __reduce_add_sync(0xffffffffu, last_items);  // only one lane holds it
+  const bool piece = decide(ib);
+  __syncwarp();  // every lane's item_pre entries are written
+  for (int a = lane; a <= nslots; a += 32) {
+    int up;
+    if (!piece) {
+      up = a < nslots ? pm.item_pre[a] : ib;
+    } else if (a < nslots) {
+      up = pm.item_pre[a] * nch_a;  // slots before a are all but the last
+    } else {
+      up = (ib - last_items) * nch_a + last_items * nch_last;
+    }
+    pm.unit_pre[a] = up;
   }
   if (lane == 0) {
     pm.item_pre[nslots] = ib;
-    pm.unit_pre[nslots] = ub;
+    pm.piece = piece;
   }
 }
 
@@ -1021,25 +1049,20 @@ __device__ void build_maps(const Params& p, const TcExtra& tx, const SlotView& s
       FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_MXFP4 || FMT == MOE_FMT_Q4_AFFINE_G64;
   const int ns = sv.U + p.has_shared;
   const int W = gridDim.x * tc_warps<FMT, NTG>();
-  auto jobs = [&](auto items_of) {  // items of the phase, by one warp
-    int J = 0;
-    for (int a = threadIdx.x & 31; a < ns; a += 32) J += items_of(a);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) J += __shfl_xor_sync(0xffffffffu, J, o);
-    return J;
-  };
   if (warp == 0) {
-    auto items = [&](int a) {
-      return (a == sv.U ? tx.tiles_s : tx.tiles_i) * ceil_div(slot_cols(p, sv, a), 8 * NTG);
-    };
-    const bool piece = tx.gu_piece != 0 && (tx.force_split != 0 || split_jobs(jobs(items), W, kFourBit));
-    build_map(ns, piece, items, [&](int) { return tx.nch_h; }, gu);
-    if ((threadIdx.x & 31) == 0) gu.piece = piece;
+    const bool may = tx.gu_piece != 0, force = tx.force_split != 0;
+    build_map(
+        ns, tx.nch_h, tx.nch_h,
+        [&](int a) {
+          return (a == sv.U ? tx.tiles_s : tx.tiles_i) * ceil_div(slot_cols(p, sv, a), 8 * NTG);
+        },
+        [&](int J) { return may && (force || split_jobs(J, W, kFourBit)); }, gu);
   } else if (warp == 1) {
-    auto items = [&](int a) { return tx.tiles_h * ceil_div(slot_cols(p, sv, a), 8 * NTG); };
-    const bool piece = tx.dn_piece != 0 && (tx.force_split != 0 || split_jobs(jobs(items), W, kFourBit));
-    build_map(ns, piece, items, [&](int a) { return a == sv.U ? tx.nch_s : tx.nch_i; }, dn);
-    if ((threadIdx.x & 31) == 0) dn.piece = piece;
+    const bool may = tx.dn_piece != 0, force = tx.force_split != 0;
+    build_map(
+        ns, tx.nch_i, p.has_shared ? tx.nch_s : tx.nch_i,
+        [&](int a) { return tx.tiles_h * ceil_div(slot_cols(p, sv, a), 8 * NTG); },
+        [&](int J) { return may && (force || split_jobs(J, W, kFourBit)); }, dn);
   }
 }
 
@@ -1072,6 +1095,9 @@ __device__ void gate_up_phase(const Params& p, const TcExtra& tx, const SlotView
     Rg.sc[3] = Ru.sc[1];
     Rg.bi[2] = Ru.bi[0];
     Rg.bi[3] = Ru.bi[1];
+    // the tensor scales now, so their round trip overlaps the job's weight stream
+    const float tsg = (FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_FP8_E4M3) ? __ldg(G.tscale + e) : 1.f;
+    const float tsu = (FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_FP8_E4M3) ? __ldg(Um.tscale + e) : 1.f;
     JobCols<NTG> C;
 #pragma unroll
     for (int q = 0; q < NTG; ++q) {
@@ -1103,8 +1129,6 @@ __device__ void gate_up_phase(const Params& p, const TcExtra& tx, const SlotView
       run_chunks<FMT, NTG, false>(Rg, C, ncols, p.h, 0, tx.nch_h, acc, sm, ring, p.x);
     }
     // epilogue: fragment f = rows g (f < 2) / g + 8, columns 2t, 2t + 1
-    const float tsg = (FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_FP8_E4M3) ? __ldg(G.tscale + e) : 1.f;
-    const float tsu = (FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_FP8_E4M3) ? __ldg(Um.tscale + e) : 1.f;
 #pragma unroll
     for (int q = 0; q < NTG; ++q)
 #pragma unroll
@@ -1205,22 +1229,50 @@ __device__ void down_phase(const Params& p, const TcExtra& tx, const SlotView& s
     old = __shfl_sync(0xffffffffu, old, 0);
     if (old + 1u != col_target) return;
     __threadfence();
-    // blend the 32 columns of tile ct for every row: lane = column
+    // blend the 32 columns of tile ct for every row: lane = column. The values of kBR rows
+    // (kBS slots each) are loaded together, one round trip to L2, then added in slot order.
     const int c = 32 * ct + lane;
     if (c >= p.h) return;
-    for (int r = 0; r < p.m; ++r) {
-      float o = 0.f;
-      for (int s2 = 0; s2 < p.k; ++s2) {
-        const int pair = r * p.k + s2;
-        const float om = p.before_ffn ? 1.f : sv.wts[pair];
-        o = fmaf(om, __ldcg(p.ypart + (size_t)sv.tp[pair] * p.h + c), o);
+    constexpr int kBR = 4, kBS = 8;
+    for (int r0 = 0; r0 < p.m; r0 += kBR) {
+      float o[kBR];
+#pragma unroll
+      for (int i = 0; i < kBR; ++i) o[i] = 0.f;
+      for (int s0 = 0; s0 < p.k; s0 += kBS) {
+        float v[kBR][kBS];
+#pragma unroll
+        for (int i = 0; i < kBR; ++i)
+#pragma unroll
+          for (int j = 0; j < kBS; ++j) {
+            const int r = r0 + i, s2 = s0 + j;
+            v[i][j] = (r < p.m && s2 < p.k)
+                          ? __ldcg(p.ypart + (size_t)sv.tp[r * p.k + s2] * p.h + c)
+                          : 0.f;
+          }
+#pragma unroll
+        for (int i = 0; i < kBR; ++i)
+#pragma unroll
+          for (int j = 0; j < kBS; ++j) {
+            const int r = r0 + i, s2 = s0 + j;
+            if (r < p.m && s2 < p.k)
+              o[i] = fmaf(p.before_ffn ? 1.f : sv.wts[r * p.k + s2], v[i][j], o[i]);
+          }
       }
-      if (p.has_shared) o = fmaf(sv.gamma[r], __ldcg(p.ysh + (size_t)r * p.h + c), o);
-      const size_t oi = (size_t)r * p.h + c;
-      if (p.out_bf16) {
-        reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
-      } else {
-        reinterpret_cast<float*>(p.out)[oi] = o;
+      float sh[kBR];
+#pragma unroll
+      for (int i = 0; i < kBR; ++i)
+        sh[i] = (p.has_shared && r0 + i < p.m) ? __ldcg(p.ysh + (size_t)(r0 + i) * p.h + c) : 0.f;
+#pragma unroll
+      for (int i = 0; i < kBR; ++i) {
+        const int r = r0 + i;
+        if (r >= p.m) break;
+        if (p.has_shared) o[i] = fmaf(sv.gamma[r], sh[i], o[i]);
+        const size_t oi = (size_t)r * p.h + c;
+        if (p.out_bf16) {
+          reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o[i]);
+        } else {
+          reinterpret_cast<float*>(p.out)[oi] = o[i];
+        }
       }
     }
   });
