@@ -202,7 +202,8 @@ TcLayout tc_layout(const moe_cfg& c, int m, size_t off) {
   }
   L.gu_slots = take(gu_bytes);
   L.dn_slots = take(dn_bytes);
-  L.tk_words = (t.j_gu_max + t.j_dn_max) * t.ncg_max + t.tiles_h;
+  // job tickets of both phases, column-tile tickets, per-slot ready counters (cap + shared)
+  L.tk_words = (t.j_gu_max + t.j_dn_max) * t.ncg_max + t.tiles_h + (int)cap + 1;
   L.tk = take((size_t)L.tk_words * 4);
 #ifdef MOE_PHASE_TIMERS
   L.stamps = take((size_t)1024 * 16 * 8);  // [CTA][16] uint64, last region of the workspace
@@ -739,6 +740,7 @@ extern "C" int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, cons
     tx.tk_gu = (unsigned*)(ws + tl.tk);
     tx.tk_dn = tx.tk_gu + (size_t)ts.j_gu_max * ts.ncg_max;
     tx.tk_col = tx.tk_dn + (size_t)ts.j_dn_max * ts.ncg_max;
+    tx.ready = tx.tk_col + ts.tiles_h;
     tx.tk_words = tl.tk_words;
     tx.stamps = tl.stamps ? (unsigned long long*)(ws + tl.stamps) : nullptr;
     tc::TcPlan pl;

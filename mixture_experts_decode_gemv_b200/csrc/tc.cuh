@@ -806,7 +806,8 @@ struct TcExtra {
   unsigned* tk_gu;     // per gate/up job: chunks finished
   unsigned* tk_dn;     // per down job: chunks finished
   unsigned* tk_col;    // per 32-column tile: down jobs finished
-  int tk_words;        // words of the three ticket arrays (zeroed at the start of every call)
+  unsigned* ready;     // per slot: gate/up jobs whose act rows are written
+  int tk_words;        // words of the ticket and ready arrays (zeroed at the start of every call)
   unsigned long long* stamps;  // phase timestamps [CTA][16] (timer builds only, else null)
 };
 
@@ -1147,14 +1148,28 @@ __device__ void gate_up_phase(const Params& p, const TcExtra& tx, const SlotView
           split_store<F16>(act_mul(p.act_kind, gv, uv), row, act_pos<FMT>(i), p.ctrl + kStatus);
         }
       }
+    // the job's act rows are written: count it for its slot (down jobs of the slot wait for all)
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      atomicAdd(tx.ready + a, 1u);
+    }
   });
 }
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+constexpr long long kChainSpinLimit = 2000000000LL;  // clock cycles (about a second)
 
 // ---- down phase + blend -----------------------------------------------------------------------
 
 template <int FMT, int NTG>
 __device__ void down_phase(const Params& p, const TcExtra& tx, const SlotView& sv,
-                           const PhaseMap& pm, int* counter, uint8_t* ring) {
+                           const PhaseMap& pm, const PhaseMap& gu, long long spin_limit,
+                           unsigned extra, int* counter, uint8_t* ring) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int U = sv.U, ns = U + p.has_shared;
   // (slot, column group) items per column tile: the blend waits for all of them
@@ -1162,6 +1177,7 @@ __device__ void down_phase(const Params& p, const TcExtra& tx, const SlotView& s
   for (int a = lane; a < ns; a += 32) col_target += (unsigned)ceil_div(slot_cols(p, sv, a), 8 * NTG);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) col_target += __shfl_xor_sync(0xffffffffu, col_target, o);
+  int ready_slot = -1;  // the last slot whose gate/up jobs this warp saw complete
   for_units(pm, ns, blockIdx.x, gridDim.x, pm.piece != 0, tc_warps<FMT, NTG>(), counter,
             [&](int a) { return a == U ? tx.nch_s : tx.nch_i; },
             [&](int a, int item, int c0, int c1, bool whole) {
@@ -1169,6 +1185,22 @@ __device__ void down_phase(const Params& p, const TcExtra& tx, const SlotView& s
     const int n = slot_cols(p, sv, a);
     const int ncg = ceil_div(n, 8 * NTG);
     const int ct = item / ncg, cg = item - ct * ncg;
+    if (a != ready_slot) {
+      // the slot's act rows: wait (bounded) until every gate/up job of the slot has counted
+      if (lane == 0) {
+        // extra: 1 in the failure-detection test (the wait then runs out), else 0
+        const unsigned want = (unsigned)(gu.item_pre[a + 1] - gu.item_pre[a]) + extra;
+        const long long t0 = clock64();
+        while (ld_acquire_u32(tx.ready + a) < want) {
+          if (clock64() - t0 > spin_limit) {
+            atomicExch(p.ctrl + kStatus, (unsigned)MOE_ERR_DEVICE_TIMEOUT);
+            break;
+          }
+        }
+      }
+      __syncwarp();
+      ready_slot = a;
+    }
     const MatDev D = pick_mat(sh, p.sd, p.rd);
     const int e = sh ? 0 : sv.slot_e[a];
     const int beg = sh ? 0 : sv.slot_beg[a];
@@ -1504,14 +1536,11 @@ __global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_fused_kernel(
     for (int r = tid; r < m; r += kThreads) p.gamma[r] = R.gamma[r];
   }
   TC_STAMP(5);
-  bar.arrive();
-  TC_STAMP(6);
-  bar.wait(2);
-  TC_STAMP(7);
   pdl_launch_dependents();
 
-  // ---- E: down + blend ------------------------------------------------------------------------
-  down_phase<FMT, NTG>(p, tx, sv, s_dn, &s_next[1], tc_ring + warp * ring_bytes<FMT, NTG>());
+  // ---- E: down + blend (each slot's down jobs start once its gate/up jobs have all counted) ---
+  down_phase<FMT, NTG>(p, tx, sv, s_dn, s_gu, pl.spin_limit, pl.bar_extra, &s_next[1],
+                       tc_ring + warp * ring_bytes<FMT, NTG>());
   TC_STAMP(11);  // warp 0's own share done
 #ifdef MOE_PHASE_TIMERS
   __syncthreads();
@@ -1633,7 +1662,9 @@ __global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_down_kernel(
   const SlotView sv = global_slots(p, slot_beg, slot_n);
   build_maps<FMT, NTG>(p, tx, sv, s_gu, s_dn, warp);
   __syncthreads();
-  down_phase<FMT, NTG>(p, tx, sv, s_dn, &s_next, tc_ring + warp * ring_bytes<FMT, NTG>());
+  // the gate/up kernel has finished (programmatic-launch wait): every slot is ready at once
+  down_phase<FMT, NTG>(p, tx, sv, s_dn, s_gu, kChainSpinLimit, 0u, &s_next,
+                       tc_ring + warp * ring_bytes<FMT, NTG>());
 }
 
 }  // namespace tc

@@ -176,6 +176,36 @@ def test_repeated_calls_are_bit_identical_and_workspace_reusable():
     assert dev.device_status(ws) == B.MOE_OK
 
 
+@pytest.mark.parametrize("name,m,path", [("qwen3_30b_a3b", 1, "auto"), ("lfm2_8b_a1b", 4, "auto"),
+                                         ("qwen3_6_35b_a3b", 16, "auto"),
+                                         ("qwen3_6_35b_a3b", 16, "chain"),
+                                         ("ragged_fp8_geglu", 40, "auto")])
+def test_no_write_outside_the_output_and_workspace(name, m, path):
+    """Canaries: the call writes nothing in the 64 KB before and after its output and workspace."""
+    cfg = SMALL.get(name) or CONFIGS[name]
+    lay, dev, _ = layer_for(cfg)
+    g = 65536  # guard bytes on each side (keeps the 256-byte alignment of both buffers)
+    nb = dev.workspace_bytes(m)
+    wbuf = torch.full((nb + 2 * g,), 0xA5, dtype=torch.uint8, device="cuda")
+    ws = wbuf[g:g + nb]
+    B.moe_workspace_init(ws, nb, torch.cuda.current_stream())
+    out0 = dev.new_out(m)
+    esz = out0.element_size()
+    obuf = torch.full((out0.numel() * esz + 2 * g,), 0x5A, dtype=torch.uint8, device="cuda")
+    out = obuf[g:g + out0.numel() * esz].view(out0.dtype).view(out0.shape)
+    x = dev.x_to_device(lay.x(m))
+    with _Path(path):
+        dev.forward(x, out, ws)
+    torch.cuda.synchronize()
+    assert dev.device_status(ws) == B.MOE_OK
+    assert bool((wbuf[:g] == 0xA5).all()) and bool((wbuf[g + nb:] == 0xA5).all())
+    assert bool((obuf[:g] == 0x5A).all()) and bool((obuf[g + out0.numel() * esz:] == 0x5A).all())
+    ref = dev.new_out(m)
+    dev.forward(x, ref, dev.new_workspace(m))
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+
+
 @pytest.mark.parametrize("m", [1, 3, 8, 40])
 def test_bf16_output_is_rounded_fp32_output(m):
     # every launch path (the persistent kernel at small m, the multi-kernel path above it)
@@ -324,9 +354,10 @@ def test_work_split_does_not_change_the_bits(name, m):
 
 
 def test_grid_barrier_timeout_is_reported_and_the_workspace_recovers():
-    """A barrier wait that runs out (made to expect one arrival too many, with a ~1 ms budget)
-    ends the launch with MOE_ERR_DEVICE_TIMEOUT in the workspace status; after
-    moe_workspace_init the same workspace gives the normal result again."""
+    """A barrier wait and the down jobs' waits for their slot's gate/up jobs that run out (made to
+    expect one arrival too many, with a ~1 ms budget) end the launch with MOE_ERR_DEVICE_TIMEOUT
+    in the workspace status; after moe_workspace_init the same workspace gives the normal
+    result again."""
     lay, dev, _ = layer_for(CONFIGS["qwen3_30b_a3b"])
     m = 1
     assert dev.launches(m) == 1
