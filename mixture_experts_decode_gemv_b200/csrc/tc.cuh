@@ -429,8 +429,10 @@ struct SlotMap {
 // the lane's live columns only. 2 to 8 stages, as many as the job's live columns leave room for.
 constexpr int kRingCtaBytes = 192 * 1024;  // dynamic shared memory per CTA: the warps' rings
 
+// Weight pieces: evict-first in L2, and a 256-byte L2 fetch on a miss, so the k-tiles that
+// follow along the same row (64 bytes each for bf16) find their bytes in L2.
 __device__ __forceinline__ void cp16_ef(uint32_t dst, const void* src, int n, uint64_t pol) {
-  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst),
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint.L2::256B [%0], [%1], 16, %2, %3;" ::"r"(dst),
                "l"(src), "r"(n), "l"(pol)
                : "memory");
 }
