@@ -47,7 +47,7 @@ SWEEP_CONFIGS = ("qwen3_30b_a3b", "lfm2_8b_a1b", "qwen3_6_35b_a3b", "llama4_scou
 # DRAM bytes (read + write) per launch of the layer's kernel, from a single-pass ncu capture of
 # the same workload (profiles/tc_fused_kernel_traffic_llama4_scout_m64.md); retaken whenever the
 # kernel changes.
-PROFILED_TRAFFIC: dict = {("llama4_scout", 64): 4.03e9 + 5.5e6}
+PROFILED_TRAFFIC: dict = {("llama4_scout", 64): 4.03e9 + 5.9e6}
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 WINDOWS = 5

@@ -916,20 +916,13 @@ struct PhaseMap {
   int piece;                    // 1: the phase's jobs are split by chunk
 };
 
-// Whether a phase of J jobs (items) runs split by chunk on a grid of W warps. Below a threshold
-// there are too few whole jobs to keep enough warps streaming: fewer than W for the 4-bit
-// formats (a k-tile costs many decode and scale instructions, so a warp's serial chain sets the
-// time), fewer than W / 2 for bf16 and FP8 (a k-tile is mostly its memory round trip, and every
-// piece restarts the warp's copy pipeline and adds a ticket). From there to W whole jobs keep
-// the grid busy. Above W, whole jobs are kept unless they leave the busiest warp more than 10%
-// above the average. Measured on the B200 with cold calls at m = 1..64 over the published shapes.
-__device__ __forceinline__ bool split_jobs(int J, int W, bool four_bit) {
-  if (J <= 0) return false;
-  if (J < (four_bit ? W : W / 2)) return true;
-  if (J < W) return false;
-  const int per = (J + W - 1) / W;  // whole jobs of the busiest warp
-  return (long long)per * W * 10 > (long long)J * 11;
-}
+// Whether a phase of J jobs (items) runs split by chunk on a grid of W warps: when there are
+// fewer whole jobs than half the warps, so that more than half the grid would idle. Above that,
+// whole jobs (handed out round-robin and taken dynamically by the CTA's warps) are balanced well
+// enough, and every piece would restart its warp's copy pipeline and add a ticket. Measured on
+// the B200 with cold calls at m = 1..64 over the published shapes, every format: the cases
+// where splitting won had J < 0.4 W, those where whole jobs won J > 0.55 W.
+__device__ __forceinline__ bool split_jobs(int J, int W) { return J > 0 && J < W / 2; }
 
 // By one warp: the prefix map of a phase over nslots slots. One scan gives the items (jobs)
 // before each slot and their total J, from which decide(J) says whether the phase splits its jobs
@@ -1048,8 +1041,6 @@ __device__ __forceinline__ int slot_cols(const Params& p, const SlotView& sv, in
 template <int FMT, int NTG>
 __device__ void build_maps(const Params& p, const TcExtra& tx, const SlotView& sv, PhaseMap& gu,
                            PhaseMap& dn, int warp) {
-  constexpr bool kFourBit =
-      FMT == MOE_FMT_NVFP4 || FMT == MOE_FMT_MXFP4 || FMT == MOE_FMT_Q4_AFFINE_G64;
   const int ns = sv.U + p.has_shared;
   const int W = gridDim.x * tc_warps<FMT, NTG>();
   if (warp == 0) {
@@ -1059,13 +1050,13 @@ __device__ void build_maps(const Params& p, const TcExtra& tx, const SlotView& s
         [&](int a) {
           return (a == sv.U ? tx.tiles_s : tx.tiles_i) * ceil_div(slot_cols(p, sv, a), 8 * NTG);
         },
-        [&](int J) { return may && (force || split_jobs(J, W, kFourBit)); }, gu);
+        [&](int J) { return may && (force || split_jobs(J, W)); }, gu);
   } else if (warp == 1) {
     const bool may = tx.dn_piece != 0, force = tx.force_split != 0;
     build_map(
         ns, tx.nch_i, p.has_shared ? tx.nch_s : tx.nch_i,
         [&](int a) { return tx.tiles_h * ceil_div(slot_cols(p, sv, a), 8 * NTG); },
-        [&](int J) { return may && (force || split_jobs(J, W, kFourBit)); }, dn);
+        [&](int J) { return may && (force || split_jobs(J, W)); }, dn);
   }
 }
 
