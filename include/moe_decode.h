@@ -175,17 +175,20 @@ int moe_decode_forward(const moe_cfg* cfg, int m, const void* x, const void* rou
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* Number of kernel launches moe_decode_forward makes for this cfg, m and weight tables on the
- * current device, into *launches: 1 when the whole call runs as one persistent kernel (m <= 4,
- * one weight format for every projection, activations within the kernel's shared memory), else
- * 3 to 5 (router, gate/up and down, the last two split when the shared expert has its own
- * format). The tables are validated as in moe_decode_forward; nothing is launched. For callers
- * that budget graph nodes or count launches; the decode pages have no counterpart. */
+ * current device, into *launches: 1 when the whole call runs as one persistent kernel (the
+ * tensor-core kernel at every m for one weight format among bf16, FP8, NVFP4, MXFP4 and Q4 with
+ * bf16 activations; the CUDA-core kernel for f32 layers with m <= 4 whose activations fit its
+ * shared memory), else 3 to 5 (router, gate/up and down, the last two split when the shared
+ * expert has its own format; 3 when moe_debug_set_path forces the multi-kernel path). The tables
+ * are validated as in moe_decode_forward; nothing is launched. For callers that budget graph
+ * nodes or count launches; the decode pages have no counterpart. */
 int moe_decode_launches(const moe_cfg* cfg, int m, const moe_expert_table* routed,
                         const moe_expert_table* shared, int* launches);
 
-/* Test aid for failure detection without a GPU fault. After this call the persistent kernel's
- * grid-barrier waits expect `extra_arrivals` (0 or 1) more arrivals than any launch makes and
- * give up after `spin_limit_cycles` SM clock cycles (0: the default budget of about a second).
+/* Test aid for failure detection without a GPU fault. After this call the persistent kernels'
+ * device-side waits (the grid barrier; in the tensor-core kernel also each down job's wait for
+ * its expert's gate/up jobs) expect `extra_arrivals` (0 or 1) more arrivals than any launch makes
+ * and give up after `spin_limit_cycles` SM clock cycles (0: the default budget of about a second).
  * Every wait stays bounded, so each launch ends; its workspace status then reads
  * MOE_ERR_DEVICE_TIMEOUT and its outputs are undefined (call moe_workspace_init before reusing
  * the workspace). moe_debug_barrier_test(0, 0) restores normal operation. Process-wide; do not
@@ -202,9 +205,10 @@ int moe_debug_set_path(int path);
 
 /* Test aid: how the tensor-core path shares out its work in every later forward call in this
  * process. mode 0 is the automatic choice; 1 gives every job (32 weight rows of one expert
- * projection) to one warp; 2 splits jobs into 256-element pieces of the reduction wherever the
- * workspace holds their partial values. The results are the same bits in every mode (the pieces'
- * values are summed in one fixed order); tests use this to check that. Process-wide; do not call
+ * projection) to one warp; 2 splits jobs into pieces of one canonical chunk of the reduction
+ * (eight k-tiles of the format) wherever the workspace holds their partial values. The results
+ * are the same bits in every mode (the pieces' values are summed in one fixed order); tests use
+ * this to check that. Process-wide; do not call
  * it while other threads run forward calls. Returns MOE_ERR_BAD_OPTION for other values. The
  * decode pages have no counterpart. */
 int moe_debug_set_split(int mode);

@@ -27,7 +27,7 @@
 // so each B fragment is one 8-byte load.
 //
 // Canonical arithmetic (the same for every m, every launch path and every work split): K is cut
-// into chunks of 256 elements. A chunk's value is the MMA chain over its k-steps starting from
+// into chunks of eight k-tiles (chunk_elems). A chunk's value is the MMA chain over its k-steps starting from
 // zero; for MXFP4 and Q4 every k-tile is its own chain from zero and is scaled into the chunk:
 //   MXFP4: chunk = fma(2^e, D_tile, chunk)
 //   Q4:    chunk = fma(16 s, D_tile, chunk); chunk = fma(b - 16 s, D_ones, chunk)
@@ -1370,18 +1370,23 @@ __device__ void tc_group(int te, TcRoute& R) {
 // ---- the persistent kernel: the whole call in one launch ------------------------------------------
 
 struct TcPlan {
-  long long spin_limit;       // clock cycles a grid-barrier wait may spin before it gives up
+  long long spin_limit;       // clock cycles a device-side wait may spin before it gives up
   long long l2_prefetch_cap;  // largest per-call down-projection byte count asked into L2
-  unsigned bar_extra;         // arrivals a barrier waits for beyond the grid (0; 1 in tests)
+  unsigned bar_extra;         // arrivals the barrier and each ready wait expect beyond the real
+                              // ones (0; 1 in the failure-detection test)
 };
 
-// Phases (all CTAs co-resident, cooperative launch, one CTA of 16 warps per SM):
+// Phases (all CTAs co-resident, cooperative launch, one CTA of 8 or 16 warps per SM):
 //   A  router logits, one warp per (router row, activation row) over the whole grid; the
-//      activations in the operand type and order; zero the call's tickets; arrive at barrier 1.
+//      activations in the operand type and order; zero the call's tickets and ready counters;
+//      arrive and wait at the grid barrier (the only one).
 //   C  every CTA routes every row and groups the pairs in its shared memory; the last warp asks
-//      L2 for this CTA's share of the active experts' down rows.
-//   D  gate/up jobs over all warps of the grid (tc::gate_up_phase); arrive and wait at barrier 2.
-//   E  down jobs over all warps; the warp completing a 32-column tile blends it (tc::down_phase).
+//      L2 for this CTA's share of the active experts' down rows; warps 0 and 1 build the two
+//      phases' maps and split decisions.
+//   D  gate/up jobs over all warps of the grid (tc::gate_up_phase); each job counts in its slot's
+//      ready counter.
+//   E  down jobs over all warps, each slot's once its ready counter is full; the warp completing
+//      a 32-column tile blends it (tc::down_phase).
 template <int FMT, int NTG>
 __global__ void __launch_bounds__(32 * tc_warps<FMT, NTG>(), 1) tc_fused_kernel(
     const __grid_constant__ Params p, const __grid_constant__ TcExtra tx,
