@@ -916,13 +916,17 @@ struct PhaseMap {
   int piece;                    // 1: the phase's jobs are split by chunk
 };
 
-// Whether a phase of J jobs (items) runs split by chunk on a grid of W warps: when there are
-// fewer whole jobs than half the warps, so that more than half the grid would idle. Above that,
-// whole jobs (handed out round-robin and taken dynamically by the CTA's warps) are balanced well
-// enough, and every piece would restart its warp's copy pipeline and add a ticket. Measured on
-// the B200 with cold calls at m = 1..64 over the published shapes, every format: the cases
-// where splitting won had J < 0.4 W, those where whole jobs won J > 0.55 W.
-__device__ __forceinline__ bool split_jobs(int J, int W) { return J > 0 && J < W / 2; }
+// Whether a phase of J jobs (items) of nch chunks each runs split by chunk on a grid of W warps:
+// when there are fewer whole jobs than half the warps (more than half the grid would idle) and a
+// job is long enough to be worth cutting: at least four chunks, or any length for the formats
+// whose k-tiles are instruction-heavy (MXFP4, Q4: decode plus a post-scaled chain per k-tile).
+// A piece restarts its warp's copy pipeline and adds a ticket, which a short bf16, FP8 or NVFP4
+// job does not win back. Above half the warps, whole jobs (handed out round-robin and taken
+// dynamically by the CTA's warps) are balanced well enough. Measured on the B200 at m = 1..64
+// over the published shapes, every format.
+__device__ __forceinline__ bool split_jobs(int J, int W, int nch, bool heavy) {
+  return J > 0 && J < W / 2 && (heavy || nch >= 4);
+}
 
 // By one warp: the prefix map of a phase over nslots slots. One scan gives the items (jobs)
 // before each slot and their total J, from which decide(J) says whether the phase splits its jobs
@@ -1041,6 +1045,7 @@ __device__ __forceinline__ int slot_cols(const Params& p, const SlotView& sv, in
 template <int FMT, int NTG>
 __device__ void build_maps(const Params& p, const TcExtra& tx, const SlotView& sv, PhaseMap& gu,
                            PhaseMap& dn, int warp) {
+  constexpr bool kHeavy = Traits<FMT>::POST;  // MXFP4, Q4
   const int ns = sv.U + p.has_shared;
   const int W = gridDim.x * tc_warps<FMT, NTG>();
   if (warp == 0) {
@@ -1050,13 +1055,13 @@ __device__ void build_maps(const Params& p, const TcExtra& tx, const SlotView& s
         [&](int a) {
           return (a == sv.U ? tx.tiles_s : tx.tiles_i) * ceil_div(slot_cols(p, sv, a), 8 * NTG);
         },
-        [&](int J) { return may && (force || split_jobs(J, W)); }, gu);
+        [&](int J) { return may && (force || split_jobs(J, W, tx.nch_h, kHeavy)); }, gu);
   } else if (warp == 1) {
     const bool may = tx.dn_piece != 0, force = tx.force_split != 0;
     build_map(
         ns, tx.nch_i, p.has_shared ? tx.nch_s : tx.nch_i,
         [&](int a) { return tx.tiles_h * ceil_div(slot_cols(p, sv, a), 8 * NTG); },
-        [&](int J) { return may && (force || split_jobs(J, W)); }, dn);
+        [&](int J) { return may && (force || split_jobs(J, W, tx.nch_i, kHeavy)); }, dn);
   }
 }
 
