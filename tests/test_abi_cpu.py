@@ -64,8 +64,9 @@ def test_version_and_status_strings():
 
 @pytest.mark.parametrize("name", list(CONFIGS))
 def test_workspace_bytes_grows_with_m(name):
+    """One workspace sized for the largest m serves every smaller m: the size never shrinks."""
     c = make_cfg(CONFIGS[name])
-    sizes = [B.moe_workspace_bytes(c, m) for m in (1, 2, 16, 64)]
+    sizes = [B.moe_workspace_bytes(c, m) for m in range(1, 65)]
     assert all(s % 256 == 0 for s in sizes)
     assert sizes == sorted(sizes)
 
